@@ -1,0 +1,242 @@
+"""Thin Python binding of libhils (include/hils.h): HiLS attention forward.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libhils.so. PyTorch supplies device memory and the stream. There
+is no CPU fallback: if the library cannot be loaded, or a tensor is not on a
+CUDA device, the call raises.
+
+    O, idx = fwd_prefill(Q, K, V, Klm, bias, head_map, S=64, W=512, topk=16)
+    O, idx = fwd_decode(Q, Kc, Vc, Klm, bias, cache_len, head_map, S, W, topk)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+__all__ = [
+    "HilsError", "lib", "library_path", "symbols", "status_string",
+    "fwd_prefill", "fwd_decode", "prefill_workspace_size",
+    "decode_workspace_size", "PrefillArgs", "DecodeArgs", "STATUS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libhils.so")
+
+STATUS = {
+    0: "HILS_OK", 1: "HILS_ERR_INVALID_ARG", 2: "HILS_ERR_UNSUPPORTED",
+    3: "HILS_ERR_MISALIGNED", 4: "HILS_ERR_WORKSPACE_TOO_SMALL",
+    5: "HILS_ERR_CUDA", 6: "HILS_ERR_DEVICE_TIMEOUT",
+    7: "HILS_ERR_DEVICE_BAD_LENGTH",
+}
+F32, BF16 = 0, 1
+
+# Every function include/hils.h declares.
+symbols = [
+    "hils_status_string", "hils_version", "hils_prefill_workspace_size",
+    "hils_decode_workspace_size", "hils_fwd_prefill", "hils_fwd_decode",
+]
+
+
+class HilsError(RuntimeError):
+    def __init__(self, code, where=""):
+        self.code = int(code)
+        super().__init__(f"{where}: {STATUS.get(self.code, self.code)}")
+
+
+_p = ctypes.c_void_p
+_i = ctypes.c_int32
+
+
+class PrefillArgs(ctypes.Structure):
+    _fields_ = [("dtype", _i), ("B", _i), ("Hq", _i), ("Hkv", _i), ("N", _i),
+                ("d", _i), ("S", _i), ("W", _i), ("K", _i),
+                ("head_map", _p), ("Q", _p), ("Qs", _p), ("Kc", _p),
+                ("V", _p), ("Klm", _p), ("bias", _p), ("O", _p), ("idx", _p),
+                ("sel_score", _p), ("workspace", _p),
+                ("workspace_bytes", ctypes.c_size_t), ("status", _p)]
+
+
+class DecodeArgs(ctypes.Structure):
+    _fields_ = [("dtype", _i), ("B", _i), ("Hq", _i), ("Hkv", _i),
+                ("Lmax", _i), ("d", _i), ("S", _i), ("W", _i), ("K", _i),
+                ("head_map", _p), ("Q", _p), ("Qs", _p), ("Kc", _p),
+                ("V", _p), ("Klm", _p), ("bias", _p), ("cache_len", _p),
+                ("O", _p), ("idx", _p), ("sel_score", _p), ("workspace", _p),
+                ("workspace_bytes", ctypes.c_size_t), ("status", _p)]
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib():
+    """The loaded libhils.so (raises if it is missing: no fallback)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(library_path):
+                raise ImportError(
+                    f"libhils.so not built ({library_path}); run "
+                    "python -m chunk_sparse_long_landmark_b200.build")
+            L = ctypes.CDLL(library_path)
+            L.hils_status_string.restype = ctypes.c_char_p
+            L.hils_status_string.argtypes = [ctypes.c_int]
+            L.hils_version.restype = ctypes.c_int32
+            for n, T in (("prefill", PrefillArgs), ("decode", DecodeArgs)):
+                f = getattr(L, f"hils_{n}_workspace_size")
+                f.restype = ctypes.c_int
+                f.argtypes = [ctypes.POINTER(T), ctypes.POINTER(ctypes.c_size_t)]
+                f = getattr(L, f"hils_fwd_{n}")
+                f.restype = ctypes.c_int
+                f.argtypes = [ctypes.POINTER(T), ctypes.c_void_p]
+            _lib = L
+    return _lib
+
+
+def status_string(code: int) -> str:
+    return lib().hils_status_string(int(code)).decode()
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _dev(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libhils needs CUDA tensors (no CPU fallback)")
+
+
+def _stream_handle(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _head_map_array(head_map, Hq):
+    hm = list(head_map)
+    arr = (ctypes.c_int32 * max(1, len(hm)))(*hm)
+    return arr
+
+
+def _prefill_struct(Q, K, V, Klm, bias, head_map, S, W, topk, Qs=None,
+                    O=None, idx=None, sel_score=None, workspace=None,
+                    status=None):
+    B, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    hm = _head_map_array(head_map, Hq)
+    a = PrefillArgs(_dtype_code(Q), B, Hq, Hkv, N, d, S, W, topk,
+                    ctypes.cast(hm, ctypes.c_void_p), _ptr(Q), _ptr(Qs),
+                    _ptr(K), _ptr(V), _ptr(Klm), _ptr(bias), _ptr(O),
+                    _ptr(idx), _ptr(sel_score), _ptr(workspace),
+                    0 if workspace is None else workspace.numel() *
+                    workspace.element_size(), _ptr(status))
+    return a, hm
+
+
+def prefill_workspace_size(Q, K, V, Klm, bias, head_map, S, W, topk,
+                           with_sel_score=False) -> int:
+    a, hm = _prefill_struct(Q, K, V, Klm, bias, head_map, S, W, topk)
+    if with_sel_score:
+        a.sel_score = 16
+    n = ctypes.c_size_t(0)
+    rc = lib().hils_prefill_workspace_size(ctypes.byref(a), ctypes.byref(n))
+    if rc:
+        raise HilsError(rc, "hils_prefill_workspace_size")
+    return int(n.value)
+
+
+def fwd_prefill(Q, K, V, Klm, bias, head_map, S, W, topk, Qs=None, out=None,
+                idx=None, sel_score=None, workspace=None, status=None,
+                stream=None):
+    """HiLS prefill forward through hils_fwd_prefill. Returns (O, idx).
+
+    Q/Qs [B,Hq,N,d], K/V [B,Hkv,N,d], Klm [B,Hkv,N//S,d] (same dtype),
+    bias [B,Hkv,N//S] float32, head_map: Hq ints. Outputs are allocated with
+    torch when not given; the workspace too (torch's caching allocator).
+    """
+    import torch
+    _dev(Q, K, V, Klm, bias, Qs, out, idx, sel_score, workspace, status)
+    B, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    if out is None:
+        out = torch.empty_like(Q)
+    if idx is None:
+        idx = torch.empty(B, Hkv, N, topk, dtype=torch.int32, device=Q.device)
+    if workspace is None:
+        n = prefill_workspace_size(Q, K, V, Klm, bias, head_map, S, W, topk,
+                                   with_sel_score=sel_score is not None)
+        workspace = torch.empty(n, dtype=torch.uint8, device=Q.device)
+    a, hm = _prefill_struct(Q, K, V, Klm, bias, head_map, S, W, topk, Qs,
+                            out, idx, sel_score, workspace, status)
+    rc = lib().hils_fwd_prefill(ctypes.byref(a), _stream_handle(stream))
+    if rc:
+        raise HilsError(rc, "hils_fwd_prefill")
+    return out, idx
+
+
+def _decode_struct(Q, K, V, Klm, bias, cache_len, head_map, S, W, topk,
+                   Qs=None, O=None, idx=None, sel_score=None, workspace=None,
+                   status=None):
+    B, Hq, d = Q.shape
+    Hkv, Lmax = K.shape[1], K.shape[2]
+    hm = _head_map_array(head_map, Hq)
+    a = DecodeArgs(_dtype_code(Q), B, Hq, Hkv, Lmax, d, S, W, topk,
+                   ctypes.cast(hm, ctypes.c_void_p), _ptr(Q), _ptr(Qs),
+                   _ptr(K), _ptr(V), _ptr(Klm), _ptr(bias), _ptr(cache_len),
+                   _ptr(O), _ptr(idx), _ptr(sel_score), _ptr(workspace),
+                   0 if workspace is None else workspace.numel() *
+                   workspace.element_size(), _ptr(status))
+    return a, hm
+
+
+def decode_workspace_size(Q, K, V, Klm, bias, cache_len, head_map, S, W,
+                          topk, with_sel_score=False) -> int:
+    a, hm = _decode_struct(Q, K, V, Klm, bias, cache_len, head_map, S, W,
+                           topk)
+    if with_sel_score:
+        a.sel_score = 16
+    n = ctypes.c_size_t(0)
+    rc = lib().hils_decode_workspace_size(ctypes.byref(a), ctypes.byref(n))
+    if rc:
+        raise HilsError(rc, "hils_decode_workspace_size")
+    return int(n.value)
+
+
+def fwd_decode(Q, K, V, Klm, bias, cache_len, head_map, S, W, topk, Qs=None,
+               out=None, idx=None, sel_score=None, workspace=None,
+               status=None, stream=None):
+    """HiLS decode step through hils_fwd_decode. Returns (O, idx).
+
+    Q/Qs [B,Hq,d]; K/V caches [B,Hkv,Lmax,d]; Klm [B,Hkv,Lmax//S,d];
+    bias [B,Hkv,Lmax//S] float32; cache_len int32 [B] on the device.
+    """
+    import torch
+    _dev(Q, K, V, Klm, bias, cache_len, Qs, out, idx, sel_score, workspace,
+         status)
+    B, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    if out is None:
+        out = torch.empty_like(Q)
+    if idx is None:
+        idx = torch.empty(B, Hkv, topk, dtype=torch.int32, device=Q.device)
+    if workspace is None:
+        n = decode_workspace_size(Q, K, V, Klm, bias, cache_len, head_map, S,
+                                  W, topk, with_sel_score=sel_score is not None)
+        workspace = torch.empty(n, dtype=torch.uint8, device=Q.device)
+    a, hm = _decode_struct(Q, K, V, Klm, bias, cache_len, head_map, S, W,
+                           topk, Qs, out, idx, sel_score, workspace, status)
+    rc = lib().hils_fwd_decode(ctypes.byref(a), _stream_handle(stream))
+    if rc:
+        raise HilsError(rc, "hils_fwd_decode")
+    return out, idx

@@ -1,0 +1,169 @@
+/*
+ * hils.h -- C ABI of the HiLS (Hierarchical Landmark Sparse) attention
+ * forward library, libhils.so (CUDA, sm_100a).
+ *
+ * The operation is the one of "Hierarchical Sparse Attention Done Right:
+ * Toward Infinite Context Modeling" (Hu et al.):
+ *   Sec. 2.1   chunks of S tokens, c(j) = floor(j/S); aligned window start
+ *              l(i) = floor((i-W+1)/S)*S; candidates C_i = {0..l(i)/S-1};
+ *              token logit s_ij = q_i.k_j/sqrt(d).
+ *   Sec. 3     surrogate score s^_ic = q^_i.k'_c/sqrt(d) + b'_c (display
+ *              after Eq. (7)); top-K chunks I_i; Z^_ic = exp s^_ic;
+ *              Z^_i = sum_{c in I_i} Z^_ic + Z_swa.
+ *   Sec. 3     hierarchical softmax (RQ2 display): for a token j of a
+ *              selected chunk, w_ij = exp(s_ij)/Z_{i,c(j)} * Z^_{i,c(j)}/Z^_i;
+ *              for a window token (l(i) <= j <= i) the chunk-level mass is
+ *              the exact window mass, so w_ij = exp(s_ij)/Z^_i.
+ *   Sec. 4.1   Q-Cal: the optional scoring query q^ enters only s^.
+ *   Sec. 4.1   GQA: per query head, chunk weights normalised over C_i;
+ *              maximum over the heads of a kv group; one top-K set per group.
+ * Output o_i = sum_j w_ij v_j over the selected chunks and the window.
+ *
+ * Conventions fixed by this library where the paper is silent:
+ *   positions are 0-based; the window starts at max(l(i), 0); C_i is empty
+ *   when l(i) <= 0 (the row is then exact causal attention); b'_c is not
+ *   scaled by 1/sqrt(d); per-head normalisation is a softmax over C_i only;
+ *   top-K ties go to the lower chunk index; when |C_i| <= K all of C_i is
+ *   selected; idx lists the selected chunks in ascending order, padded -1.
+ *
+ * Layouts: every tensor is dense, row-major, with the innermost dimension
+ * contiguous, in the order given below. Q, Qs, K, V, landmark keys and O
+ * share one element type (hils_dtype); bias and sel_score are float32; idx
+ * and cache_len are int32. All tensor pointers are DEVICE pointers except
+ * head_map, which is a HOST array read during the call.
+ *
+ * Ownership: the caller owns every buffer, including the workspace; the
+ * library allocates no memory and keeps no state between calls other than
+ * a per-device cache of kernel attributes.
+ *
+ * Streams and errors: calls enqueue work on `stream` (a cudaStream_t, NULL
+ * = legacy default stream) and return without synchronising. Argument
+ * errors are detected on the host before any launch and returned as a
+ * hils_status; nothing is enqueued in that case. A failed launch returns
+ * HILS_ERR_CUDA. Errors found on the device (a cache_len out of range, a
+ * bounded wait that gave up) are written to *status (a device int32 the
+ * caller zeroes and reads after synchronising; NULL disables reporting);
+ * the affected outputs are then unspecified.
+ *
+ * Determinism: no floating-point atomics; repeated calls with the same
+ * inputs give bitwise identical outputs.
+ */
+#ifndef HILS_H
+#define HILS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HILS_OK = 0,
+    HILS_ERR_INVALID_ARG = 1,       /* null pointer, bad size, bad head_map */
+    HILS_ERR_UNSUPPORTED = 2,       /* valid but outside the supported set */
+    HILS_ERR_MISALIGNED = 3,        /* a tensor pointer not 16-byte aligned */
+    HILS_ERR_WORKSPACE_TOO_SMALL = 4,
+    HILS_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed */
+    HILS_ERR_DEVICE_TIMEOUT = 6,    /* device-side bounded wait gave up */
+    HILS_ERR_DEVICE_BAD_LENGTH = 7  /* device-side: cache_len outside [1, Lmax] */
+} hils_status;
+
+typedef enum { HILS_F32 = 0, HILS_BF16 = 1 } hils_dtype;
+
+/* Limits of this build (checked on the host). */
+#define HILS_MAX_HEAD_DIM 128       /* d in {64, 128} for bf16; d <= 128, d % 4 == 0 for f32 */
+#define HILS_MAX_TOPK 64            /* 1 <= K <= 64 */
+#define HILS_MAX_GROUP 16           /* G = Hq/Hkv <= 16 */
+
+/*
+ * Prefill: every position i in [0, N) of B sequences is a query.
+ *   Q, Qs  [B, Hq, N, d]   query; Qs = scoring query q^ (NULL: use Q)
+ *   Kc, V  [B, Hkv, N, d]  keys, values
+ *   Klm    [B, Hkv, nC, d] landmark keys k'_c, nC = floor(N/S)
+ *   bias   [B, Hkv, nC]    chunk bias b'_c (float32)
+ *   O      [B, Hq, N, d]   output (written)
+ *   idx    [B, Hkv, N, K]  selected chunks per (row, kv group) (written)
+ *   sel_score [B, Hq, N, K] float32: s^ of each selected chunk for every
+ *          query head, in idx order, NaN on padding (written; may be NULL,
+ *          then the workspace holds it)
+ *   head_map [Hq] HOST: kv head of each query head; every kv head must be
+ *          used by exactly G = Hq/Hkv query heads.
+ * Sizes: B, Hq, Hkv, N >= 1; S >= 1; W >= 1; 1 <= K <= HILS_MAX_TOPK.
+ */
+typedef struct {
+    int32_t dtype;                  /* hils_dtype */
+    int32_t B, Hq, Hkv, N, d, S, W, K;
+    const int32_t *head_map;        /* host [Hq] */
+    const void *Q, *Qs, *Kc, *V, *Klm;
+    const float *bias;
+    void *O;
+    int32_t *idx;
+    float *sel_score;               /* nullable */
+    void *workspace;                /* device, >= hils_prefill_workspace_size */
+    size_t workspace_bytes;
+    int32_t *status;                /* device, nullable */
+} hils_prefill_args;
+
+/*
+ * Decode: one query per sequence, the last cached token i = cache_len[b]-1,
+ * whose own key and value are already in the cache.
+ *   Q, Qs  [B, Hq, d]          query; Qs = scoring query (NULL: use Q)
+ *   Kc, V  [B, Hkv, Lmax, d]   caches
+ *   Klm    [B, Hkv, Lmax/S, d] landmark keys of the complete chunks
+ *   bias   [B, Hkv, Lmax/S]    float32
+ *   cache_len [B] DEVICE int32, each in [1, Lmax]
+ *   O      [B, Hq, d]          output (written)
+ *   idx    [B, Hkv, K]         selected chunks (written)
+ *   sel_score [B, Hq, K]       float32, nullable
+ */
+typedef struct {
+    int32_t dtype;
+    int32_t B, Hq, Hkv, Lmax, d, S, W, K;
+    const int32_t *head_map;        /* host [Hq] */
+    const void *Q, *Qs, *Kc, *V, *Klm;
+    const float *bias;
+    const int32_t *cache_len;       /* device [B] */
+    void *O;
+    int32_t *idx;
+    float *sel_score;               /* nullable */
+    void *workspace;
+    size_t workspace_bytes;
+    int32_t *status;                /* device, nullable */
+} hils_decode_args;
+
+/* Human-readable name of a status code (static string). */
+const char *hils_status_string(hils_status s);
+
+/* Library version, as 10000*major + 100*minor + patch. */
+int32_t hils_version(void);
+
+/*
+ * Workspace bytes a call with these arguments needs (only the shape fields,
+ * dtype, head_map and the nullness of sel_score are read). Writes *bytes and
+ * returns HILS_OK, or an argument error without writing.
+ */
+hils_status hils_prefill_workspace_size(const hils_prefill_args *args,
+                                        size_t *bytes);
+hils_status hils_decode_workspace_size(const hils_decode_args *args,
+                                       size_t *bytes);
+
+/*
+ * HiLS prefill forward (Sec. 2.1, Sec. 3, Sec. 4.1): landmark scoring with
+ * the causal candidate mask, per-group top-K, intra-chunk and window softmax
+ * attention, chunk-level softmax fusion. Enqueued on `stream`.
+ */
+hils_status hils_fwd_prefill(const hils_prefill_args *args, void *stream);
+
+/*
+ * HiLS decode forward: the same computation for the last query of each
+ * sequence, reading the caches. Enqueued on `stream`; graph-capturable (no
+ * host synchronisation, cache_len read on the device).
+ */
+hils_status hils_fwd_decode(const hils_decode_args *args, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HILS_H */

@@ -68,7 +68,7 @@ def load_library(path):
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
         ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
-        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     lib.oracle_max_threads.restype = ctypes.c_int
     return lib
 
@@ -148,6 +148,7 @@ class _Bound:
         idx = np.zeros((n, K), dtype=np.int32)
         shat = np.zeros((n, G, K), dtype=np.float64)
         gap = np.zeros((n,), dtype=np.float64)
+        akth = np.zeros((n,), dtype=np.float64)
         lse = np.zeros((n, G), dtype=np.float64)
         imp = None
         if imposed_idx is not None:
@@ -156,10 +157,11 @@ class _Bound:
         fails = lib.oracle_rows(ctypes.byref(self.p), n, _ptr(rb), _ptr(rg),
                                 _ptr(ri), _ptr(rr), int(score_mode), _ptr(imp),
                                 _ptr(O), _ptr(idx), _ptr(shat), _ptr(gap),
-                                _ptr(lse), int(threads))
+                                _ptr(akth), _ptr(lse), int(threads))
         if fails:
             raise RuntimeError(f"oracle failed on {fails} rows")
-        return dict(O=O, idx=idx, shat_sel=shat, gap=gap, lse=lse)
+        return dict(O=O, idx=idx, shat_sel=shat, gap=gap, akth=akth,
+                    lse=lse)
 
 
 def group_heads(head_map, g):
@@ -172,7 +174,8 @@ def prefill_rows(inp, rows, score_mode=SCORE_LANDMARK, imposed_idx=None,
 
     inp: dict from ``synth.make_prefill`` (Q, Qs, K, V, Klm, bias, head_map,
     shape). rows: int array [n, 3] of (b, g, i). Returns per-row arrays:
-    O [n,G,d] (float64), idx [n,K], shat_sel [n,G,K], gap [n], lse [n,G].
+    O [n,G,d] (float64), idx [n,K], shat_sel [n,G,K], gap [n], akth [n]
+    (a_(K), the lowest selected group score), lse [n,G].
     """
     sh = inp["shape"]
     bd = bound or _Bound(inp["Q"], inp.get("Qs"), inp["K"], inp["V"],
@@ -209,16 +212,18 @@ def scatter_prefill(inp, rows, r):
     shat = np.full((sh.B, sh.Hq, sh.N, sh.K), np.nan)
     idx = np.full((sh.B, sh.Hkv, sh.N, sh.K), -2, dtype=np.int32)
     gap = np.full((sh.B, sh.Hkv, sh.N), np.nan)
+    akth = np.full((sh.B, sh.Hkv, sh.N), np.nan)
     for g in range(sh.Hkv):
         heads = group_heads(hm, g)
         m = rows[:, 1] == g
         b, i = rows[m, 0], rows[m, 2]
         idx[b, g, i] = r["idx"][m]
         gap[b, g, i] = r["gap"][m]
+        akth[b, g, i] = r["akth"][m]
         for hh, h in enumerate(heads):
             O[b, h, i] = r["O"][m, hh]
             shat[b, h, i] = r["shat_sel"][m, hh]
-    return dict(O=O, idx=idx, shat_sel=shat, gap=gap)
+    return dict(O=O, idx=idx, shat_sel=shat, gap=gap, akth=akth)
 
 
 def decode(inp, score_mode=SCORE_LANDMARK, imposed_idx=None, threads=0,
@@ -226,7 +231,7 @@ def decode(inp, score_mode=SCORE_LANDMARK, imposed_idx=None, threads=0,
     """Oracle for one decode step: query i = cache_len[b]-1 of each sequence.
 
     Returns O [B,Hq,d] float64, idx [B,Hkv,K], shat_sel [B,Hq,K],
-    gap [B,Hkv], lse [B,Hq]. ``batches`` restricts the evaluated sequences
+    gap [B,Hkv], akth [B,Hkv], lse [B,Hq]. ``batches`` restricts the evaluated sequences
     (others are left NaN / -2). ``imposed_idx``: [B,Hkv,K] or None.
     """
     sh = inp["shape"]
@@ -250,13 +255,49 @@ def decode(inp, score_mode=SCORE_LANDMARK, imposed_idx=None, threads=0,
     lse = np.full((B, sh.Hq), np.nan)
     idx = np.full((B, Hkv, K), -2, dtype=np.int32)
     gap = np.full((B, Hkv), np.nan)
+    akth = np.full((B, Hkv), np.nan)
     hm = inp["head_map"]
     for n in range(len(rb)):
         b, g = rb[n], rg[n]
         idx[b, g] = r["idx"][n]
         gap[b, g] = r["gap"][n]
+        akth[b, g] = r["akth"][n]
         for hh, h in enumerate(group_heads(hm, g)):
             O[b, h] = r["O"][n, hh]
             shat[b, h] = r["shat_sel"][n, hh]
             lse[b, h] = r["lse"][n, hh]
-    return dict(O=O, idx=idx, shat_sel=shat, gap=gap, lse=lse)
+    return dict(O=O, idx=idx, shat_sel=shat, gap=gap, akth=akth, lse=lse)
+
+
+def prefill_at(inp, positions, score_mode=SCORE_LANDMARK, imposed_idx=None,
+               threads=0):
+    """Oracle at chosen query positions of a (possibly huge) prefill problem.
+
+    Only the Q / Qs rows at ``positions`` are copied to the host; K, V, Klm
+    and bias are copied whole. Returns per-(b, g, position) arrays shaped
+    O [B,Hkv,P,G,d], idx [B,Hkv,P,K], shat_sel [B,Hkv,P,G,K], gap/akth
+    [B,Hkv,P]. ``imposed_idx``: [B,Hkv,P,K] or None.
+    """
+    import torch
+    sh = inp["shape"]
+    pos = np.asarray(positions, dtype=np.int64)
+    P = len(pos)
+    pt = torch.as_tensor(pos, device=inp["Q"].device)
+    Qsub = inp["Q"].index_select(2, pt)
+    Qssub = inp["Qs"].index_select(2, pt) if inp.get("Qs") is not None \
+        else None
+    bd = _Bound(Qsub, Qssub, inp["K"], inp["V"], inp["Klm"], inp["bias"],
+                inp["head_map"], sh.S, sh.W, sh.K, q_rows=P)
+    bb, gg, pp = np.meshgrid(np.arange(sh.B), np.arange(sh.Hkv),
+                             np.arange(P), indexing="ij")
+    rb, rg, rp = bb.ravel(), gg.ravel(), pp.ravel()
+    imp = None
+    if imposed_idx is not None:
+        imp = np.asarray(imposed_idx, dtype=np.int32).reshape(-1, sh.K)
+    r = bd.rows(rb, rg, pos[rp], rp, score_mode, imp, threads)
+    G, d, K = sh.G, sh.d, sh.K
+    return dict(O=r["O"].reshape(sh.B, sh.Hkv, P, G, d),
+                idx=r["idx"].reshape(sh.B, sh.Hkv, P, K),
+                shat_sel=r["shat_sel"].reshape(sh.B, sh.Hkv, P, G, K),
+                gap=r["gap"].reshape(sh.B, sh.Hkv, P),
+                akth=r["akth"].reshape(sh.B, sh.Hkv, P))

@@ -145,13 +145,15 @@ static int int_cmp(const void *x, const void *y) {
  *   imposed_idx  NULL, or K chunk indices (ascending, -1 padded) to use
  *                instead of the selection (scores are still computed)
  * Outputs: O[G*d], idx[K], shat_sel[G*K] (s^ of the selected chunks, in idx
- * order; NAN for padding), gap (a_(K) - a_(K+1) or +inf), lse[G].
+ * order; NAN for padding), gap (a_(K) - a_(K+1) or +inf), akth (a_(K), the
+ * lowest selected group score, -inf if none), lse[G].
  * Returns 0, or -1 on allocation failure / bad imposed index.
  */
 static int oracle_one(const oracle_problem *p, int b, int g, int64_t i, int r,
                       const int *heads, int G, int score_mode,
                       const int32_t *imposed_idx, double *O, int32_t *idx,
-                      double *shat_sel, double *gap, double *lse) {
+                      double *shat_sel, double *gap, double *akth,
+                      double *lse) {
     const int S = p->S, d = p->d, K = p->K;
     /* [2.1] aligned window and candidate set */
     int64_t lq = floordiv(i - p->W + 1, S);
@@ -196,6 +198,7 @@ static int oracle_one(const oracle_problem *p, int b, int g, int64_t i, int r,
     qsort(cs, (size_t)nc, sizeof(cand), cand_cmp);
     int nsel = (int)(nc < K ? nc : K);
     *gap = (nc > K) ? cs[K - 1].a - cs[K].a : INFINITY;
+    *akth = nsel > 0 ? cs[nsel - 1].a : -INFINITY;
     if (imposed_idx) {
         nsel = 0;
         for (int k = 0; k < K; ++k) {
@@ -268,14 +271,14 @@ static int oracle_one(const oracle_problem *p, int b, int g, int64_t i, int r,
  * Evaluate nrows (b, g, i, r) rows: b batch, g kv head, i query position,
  * r row of Q holding that query. Outputs are row-major per row:
  *   O [nrows, G, d]  idx [nrows, K]  shat_sel [nrows, G, K]  gap [nrows]
- *   lse [nrows, G]
+ *   akth [nrows]  lse [nrows, G]
  * imposed_idx: NULL or [nrows, K]. Returns 0, or the count of failed rows.
  */
 int oracle_rows(const oracle_problem *p, int64_t nrows, const int32_t *rb,
                 const int32_t *rg, const int64_t *ri, const int32_t *rr,
                 int score_mode, const int32_t *imposed_idx, double *O,
-                int32_t *idx, double *shat_sel, double *gap, double *lse,
-                int nthreads) {
+                int32_t *idx, double *shat_sel, double *gap, double *akth,
+                double *lse, int nthreads) {
     int G = p->Hq / p->Hkv;
     int fails = 0;
 #ifdef _OPENMP
@@ -295,7 +298,7 @@ int oracle_rows(const oracle_problem *p, int64_t nrows, const int32_t *rb,
                             imposed_idx ? imposed_idx + n * p->K : NULL,
                             O + n * (int64_t)G * p->d, idx + n * p->K,
                             shat_sel + n * (int64_t)G * p->K, gap + n,
-                            lse + n * G);
+                            akth + n, lse + n * G);
         if (rc) fails++;
     }
     return fails;

@@ -1,0 +1,160 @@
+"""Host-only checks of the C ABI: the library loads, exports every function
+include/hils.h declares, and rejects bad arguments before launching anything.
+No GPU work is done here (every call below fails validation on the host or
+only sizes the workspace)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import chunk_sparse_long_landmark_b200 as hils
+from chunk_sparse_long_landmark_b200 import build as hbuild
+
+HDR = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include",
+                   "hils.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    hbuild.build()
+    return hils.lib()
+
+
+def header_functions():
+    txt = open(HDR).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(hils_[a-z_0-9]+)\s*\(", txt)))
+
+
+def test_header_symbols_exported(L):
+    names = header_functions()
+    assert names, "no functions parsed from include/hils.h"
+    assert sorted(hils.symbols) == names
+    for n in names:
+        assert hasattr(L, n), f"libhils.so does not export {n}"
+
+
+def test_status_strings(L):
+    for code, name in hils.STATUS.items():
+        assert hils.status_string(code) == name
+    assert hils.status_string(99) == "HILS_ERR_UNKNOWN"
+    assert L.hils_version() >= 100
+
+
+def _pf(**kw):
+    hm = (ctypes.c_int32 * 32)(*[h // 4 for h in range(32)])
+    base = dict(dtype=1, B=1, Hq=32, Hkv=8, N=4096, d=128, S=64, W=512, K=16,
+                head_map=ctypes.cast(hm, ctypes.c_void_p).value)
+    fake = 1 << 40                               # never dereferenced
+    ptrs = dict(Q=fake, Kc=fake + 4096, V=fake + 8192, Klm=fake + 12288,
+                bias=fake + 16384, O=fake + 20480, idx=fake + 24576,
+                workspace=fake + 28672, workspace_bytes=1 << 40)
+    base.update(ptrs)
+    base.update(kw)
+    a = hils.PrefillArgs()
+    for k, v in base.items():
+        setattr(a, k, v)
+    return a, hm
+
+
+def _ws(L, a):
+    n = ctypes.c_size_t(0)
+    rc = L.hils_prefill_workspace_size(ctypes.byref(a), ctypes.byref(n))
+    return rc, n.value
+
+
+def test_workspace_size_valid(L):
+    a, hm = _pf()
+    rc, n = _ws(L, a)
+    assert rc == 0 and n >= 4 * 32 * 4096 * 16     # s^ of selected chunks
+    a2, hm2 = _pf(sel_score=1 << 41)
+    rc2, n2 = _ws(L, a2)
+    assert rc2 == 0 and n2 < n
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("dtype", 7, 1), ("B", 0, 1), ("Hq", 0, 1), ("N", 0, 1), ("S", 0, 1),
+    ("W", 0, 1), ("K", 0, 1), ("K", 65, 2), ("Hkv", 5, 1), ("d", 256, 2),
+    ("d", 12, 2), ("head_map", 0, 1),
+])
+def test_workspace_size_rejects(L, field, value, code):
+    a, hm = _pf(**{field: value})
+    rc, _ = _ws(L, a)
+    assert rc == code, (field, value, hils.STATUS.get(rc))
+
+
+def test_bad_head_map_rejected(L):
+    hm = (ctypes.c_int32 * 32)(*([0] * 5 + [h // 4 for h in range(5, 32)]))
+    a, _ = _pf(head_map=ctypes.cast(hm, ctypes.c_void_p).value)
+    rc, _ = _ws(L, a)
+    assert rc == 1
+    hm2 = (ctypes.c_int32 * 32)(*([9] + [h // 4 for h in range(1, 32)]))
+    a2, _ = _pf(head_map=ctypes.cast(hm2, ctypes.c_void_p).value)
+    assert _ws(L, a2)[0] == 1
+
+
+@pytest.mark.parametrize("field", ["Q", "Kc", "V", "O", "idx", "bias", "Klm"])
+def test_fwd_prefill_rejects_null(L, field):
+    a, hm = _pf(**{field: 0})
+    assert L.hils_fwd_prefill(ctypes.byref(a), None) == 1
+
+
+@pytest.mark.parametrize("field", ["Q", "Kc", "V", "O", "idx", "Klm",
+                                   "workspace"])
+def test_fwd_prefill_rejects_misaligned(L, field):
+    a, hm = _pf()
+    setattr(a, field, getattr(a, field) + 8)
+    assert L.hils_fwd_prefill(ctypes.byref(a), None) == 3
+
+
+def test_fwd_prefill_rejects_small_workspace(L):
+    a, hm = _pf(workspace_bytes=1024)
+    assert L.hils_fwd_prefill(ctypes.byref(a), None) == 4
+
+
+def test_fwd_prefill_null_args(L):
+    assert L.hils_fwd_prefill(None, None) == 1
+    n = ctypes.c_size_t(0)
+    assert L.hils_prefill_workspace_size(None, ctypes.byref(n)) == 1
+    a, hm = _pf()
+    assert L.hils_prefill_workspace_size(ctypes.byref(a), None) == 1
+
+
+def _df(**kw):
+    hm = (ctypes.c_int32 * 32)(*[h // 4 for h in range(32)])
+    fake = 1 << 40
+    base = dict(dtype=1, B=8, Hq=32, Hkv=8, Lmax=8192, d=128, S=64, W=512,
+                K=32, head_map=ctypes.cast(hm, ctypes.c_void_p).value,
+                Q=fake, Kc=fake + 4096, V=fake + 8192, Klm=fake + 12288,
+                bias=fake + 16384, cache_len=fake + 20480, O=fake + 24576,
+                idx=fake + 28672, workspace=fake + 32768,
+                workspace_bytes=1 << 40)
+    base.update(kw)
+    a = hils.DecodeArgs()
+    for k, v in base.items():
+        setattr(a, k, v)
+    return a, hm
+
+
+def test_decode_validation(L):
+    a, hm = _df()
+    n = ctypes.c_size_t(0)
+    assert L.hils_decode_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert n.value > 0
+    a, hm = _df(cache_len=0)
+    assert L.hils_fwd_decode(ctypes.byref(a), None) == 1
+    a, hm = _df(Q=(1 << 40) + 4)
+    assert L.hils_fwd_decode(ctypes.byref(a), None) == 3
+    a, hm = _df(workspace_bytes=16)
+    assert L.hils_fwd_decode(ctypes.byref(a), None) == 4
+    a, hm = _df(Lmax=0)
+    assert L.hils_fwd_decode(ctypes.byref(a), None) == 1
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    Q = torch.zeros(1, 1, 8, 64)
+    with pytest.raises(ValueError):
+        hils.fwd_prefill(Q, Q, Q, Q[:, :, :1], torch.zeros(1, 1, 1), [0], 8,
+                         8, 1)

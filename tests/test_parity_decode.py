@@ -1,0 +1,93 @@
+"""GPU parity of hils_fwd_decode (through the C ABI) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import chunk_sparse_long_landmark_b200 as hils
+import synth
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def run_decode(inp, status=None):
+    sh = inp["shape"]
+    O, idx = hils.fwd_decode(inp["Q"], inp["K"], inp["V"], inp["Klm"],
+                             inp["bias"], inp["cache_len"], inp["head_map"],
+                             sh.S, sh.W, sh.K, status=status)
+    torch.cuda.synchronize()
+    return O, idx
+
+
+CASES = {
+    "f32_ragged": (synth.Shape("f32", 3, 4, 2, 64, 2048, 64, 128, 5), [2048, 1000, 70]),
+    "bf16_ragged": (synth.Shape("bf16", 4, 32, 8, 128, 16384, 64, 512, 32), [16384, 9999, 600, 1]),
+    "bf16_short": (synth.Shape("bf16", 2, 8, 2, 128, 4096, 64, 512, 32), [513, 575]),
+    "bf16_d64_S128": (synth.Shape("bf16", 2, 8, 1, 64, 8192, 128, 300, 16), [8192, 5000]),
+    "bf16_k64_g16": (synth.Shape("bf16", 1, 16, 1, 128, 32768, 64, 512, 64), [32768]),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_decode_small(name, cuda_device):
+    sh, lens = CASES[name]
+    inp = synth.make_decode(sh, seed=202, device=cuda_device, cache_len=lens)
+    O, idx = run_decode(inp)
+    parity.check_decode(inp, O, idx)
+
+
+def test_decode_config4_full(cuda_device):
+    """Batch of 8 sequences with 512K-token caches, every sequence checked."""
+    sh = synth.DECODE_CONFIGS[4]
+    inp = synth.make_decode(sh, seed=synth.seed_for(4), device=cuda_device)
+    O, idx = run_decode(inp)
+    for b in range(sh.B):                       # oracle one sequence at a time
+        sub = dict(inp, Q=inp["Q"][b:b + 1], K=inp["K"][b:b + 1],
+                   V=inp["V"][b:b + 1], Klm=inp["Klm"][b:b + 1],
+                   bias=inp["bias"][b:b + 1],
+                   cache_len=inp["cache_len"][b:b + 1],
+                   shape=sh.with_(B=1))
+        parity.check_decode(sub, O[b:b + 1], idx[b:b + 1])
+
+
+def test_decode_bad_length_reported(cuda_device):
+    """A cache_len outside [1, Lmax] is reported in the status word."""
+    sh = synth.Shape("bf16", 2, 8, 2, 128, 2048, 64, 256, 8)
+    inp = synth.make_decode(sh, seed=3, device=cuda_device,
+                            cache_len=[2048, 4096])
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    O, idx = run_decode(inp, status=st)
+    assert int(st.item()) == 7          # HILS_ERR_DEVICE_BAD_LENGTH
+    # the valid sequence is still computed correctly
+    sub = dict(inp, Q=inp["Q"][:1], K=inp["K"][:1], V=inp["V"][:1],
+               Klm=inp["Klm"][:1], bias=inp["bias"][:1],
+               cache_len=inp["cache_len"][:1], shape=sh.with_(B=1))
+    parity.check_decode(sub, O[:1], idx[:1])
+
+
+def test_decode_deterministic_and_graph(cuda_device):
+    sh = synth.Shape("bf16", 4, 32, 8, 128, 65536, 64, 512, 32)
+    inp = synth.make_decode(sh, seed=9, device=cuda_device)
+    O1, i1 = run_decode(inp)
+    O = torch.empty_like(O1)
+    idx = torch.empty_like(i1)
+    ws = torch.empty(hils.decode_workspace_size(
+        inp["Q"], inp["K"], inp["V"], inp["Klm"], inp["bias"],
+        inp["cache_len"], inp["head_map"], sh.S, sh.W, sh.K),
+        dtype=torch.uint8, device=cuda_device)
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        hils.fwd_decode(inp["Q"], inp["K"], inp["V"], inp["Klm"],
+                        inp["bias"], inp["cache_len"], inp["head_map"], sh.S,
+                        sh.W, sh.K, out=O, idx=idx, workspace=ws, stream=s)
+    s.synchronize()
+    with torch.cuda.graph(g, stream=s):
+        hils.fwd_decode(inp["Q"], inp["K"], inp["V"], inp["Klm"],
+                        inp["bias"], inp["cache_len"], inp["head_map"], sh.S,
+                        sh.W, sh.K, out=O, idx=idx, workspace=ws, stream=s)
+    O.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(O, O1) and torch.equal(idx, i1)
+    del g

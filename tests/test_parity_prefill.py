@@ -1,0 +1,118 @@
+"""GPU parity of hils_fwd_prefill (through the C ABI) against the fp64 oracle.
+
+Small problems are compared on every row; the full-size workloads of the
+scope table on edge + random rows (oracle row by row), in the same launch
+configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import chunk_sparse_long_landmark_b200 as hils
+import synth
+from tests import parity
+
+pytestmark = pytest.mark.gpu
+
+
+def run_prefill(inp, sel=False):
+    sh = inp["shape"]
+    sel_t = None
+    if sel:
+        sel_t = torch.empty(sh.B, sh.Hq, sh.N, sh.K, dtype=torch.float32,
+                            device=inp["Q"].device)
+    O, idx = hils.fwd_prefill(inp["Q"], inp["K"], inp["V"], inp["Klm"],
+                              inp["bias"], inp["head_map"], sh.S, sh.W, sh.K,
+                              Qs=inp["Qs"], sel_score=sel_t)
+    torch.cuda.synchronize()
+    return O, idx, sel_t
+
+
+SMALL = {
+    # name: (Shape, head_map or None)
+    "f32_ragged_gqa": (synth.Shape("f32", 2, 4, 2, 64, 1000, 64, 100, 5), [1, 0, 0, 1]),
+    "f32_mha_W1": (synth.Shape("f32", 1, 2, 2, 32, 300, 16, 1, 3), None),
+    "f32_topk_gt_candidates": (synth.Shape("f32", 1, 2, 1, 64, 512, 32, 64, 64), None),
+    "bf16_g4_d128": (synth.Shape("bf16", 2, 8, 2, 128, 3000, 64, 256, 8), None),
+    "bf16_d64_S128": (synth.Shape("bf16", 1, 8, 2, 64, 2500, 128, 300, 6), None),
+    "bf16_qcal": (synth.Shape("bf16", 1, 8, 2, 128, 2048, 64, 200, 4, "qcal"), None),
+    "bf16_temperature": (synth.Shape("bf16", 1, 8, 2, 128, 4096, 64, 512, 16, "temperature"), None),
+    "bf16_needles": (synth.Shape("bf16", 1, 8, 2, 128, 4096, 64, 512, 16, "needles", n_needles=4), None),
+    "bf16_g1": (synth.Shape("bf16", 1, 4, 4, 128, 1500, 64, 128, 8), None),
+    "bf16_g8": (synth.Shape("bf16", 1, 16, 2, 128, 1500, 64, 128, 8), None),
+    "bf16_g16_k64": (synth.Shape("bf16", 1, 16, 1, 64, 6000, 64, 64, 64), None),
+    "bf16_k1": (synth.Shape("bf16", 1, 4, 1, 128, 1200, 64, 64, 1), None),
+    "bf16_no_candidates": (synth.Shape("bf16", 1, 4, 1, 128, 200, 64, 512, 4), None),
+    "bf16_single_token": (synth.Shape("bf16", 1, 4, 1, 128, 1, 64, 16, 2), None),
+    "bf16_ragged_tail": (synth.Shape("bf16", 1, 8, 2, 128, 2111, 64, 190, 7), [0, 1, 0, 1, 0, 1, 0, 1]),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_prefill_small(name, cuda_device):
+    sh, hm = SMALL[name]
+    inp = synth.make_prefill(sh, seed=101, device=cuda_device, head_map=hm)
+    O, idx, sel = run_prefill(inp, sel=True)
+    parity.check_prefill(inp, O, idx, sel_gpu=sel)
+
+
+def test_config1_full(cuda_device):
+    sh = synth.PREFILL_CONFIGS[1]
+    inp = synth.make_prefill(sh, seed=synth.seed_for(1), device=cuda_device)
+    O, idx, sel = run_prefill(inp, sel=True)
+    parity.check_prefill(inp, O, idx, sel_gpu=sel)
+
+
+def test_exact_landmarks_full_topk_is_causal_attention(cuda_device):
+    """Chunks of identical keys with (k', b') = (k̄, log S) and K >= |C_i|:
+    the result must be plain causal attention (checked against torch SDPA
+    in float64, an independent routine)."""
+    sh = synth.Shape("bf16", 1, 8, 2, 128, 1024, 64, 128, 64, "exact")
+    inp = synth.make_prefill(sh, seed=5, device=cuda_device)
+    O, idx, _ = run_prefill(inp)
+    hm = inp["head_map"]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        inp["Q"].double(), inp["K"][:, hm].double(), inp["V"][:, hm].double(),
+        is_causal=True)
+    err = (O.double() - ref).abs().max().item()
+    assert err <= parity.BF16_ABS, err
+
+
+def test_deterministic(cuda_device):
+    sh = synth.Shape("bf16", 1, 8, 2, 128, 4096, 64, 512, 16)
+    inp = synth.make_prefill(sh, seed=3, device=cuda_device)
+    O1, i1, _ = run_prefill(inp)
+    O2, i2, _ = run_prefill(inp)
+    assert torch.equal(O1, O2) and torch.equal(i1, i2)
+
+
+def test_user_stream(cuda_device):
+    sh = synth.Shape("bf16", 1, 8, 2, 128, 2048, 64, 256, 8)
+    inp = synth.make_prefill(sh, seed=4, device=cuda_device)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        O, idx = hils.fwd_prefill(inp["Q"], inp["K"], inp["V"], inp["Klm"],
+                                  inp["bias"], inp["head_map"], sh.S, sh.W,
+                                  sh.K, stream=s)
+    s.synchronize()
+    parity.check_prefill(inp, O, idx, positions=parity.sample_positions(sh))
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 5])
+def test_full_size_config_sampled(cfg, cuda_device):
+    sh = synth.PREFILL_CONFIGS[cfg]
+    inp = synth.make_prefill(sh, seed=synth.seed_for(cfg), device=cuda_device)
+    O, idx, sel = run_prefill(inp, sel=True)
+    pos = parity.sample_positions(sh, n_random=40, seed=cfg)
+    stats = parity.check_prefill(inp, O, idx, positions=pos, sel_gpu=sel)
+    assert stats["rows"] >= len(pos) * sh.Hkv
+    # every row's idx is ascending, in C_i, -1 padded (all rows, on device)
+    i = torch.arange(sh.N, device=cuda_device)
+    nc = torch.clamp(torch.div(i - sh.W + 1, sh.S, rounding_mode="floor"),
+                     min=0)
+    valid = idx >= 0
+    assert bool((idx < nc.view(1, 1, -1, 1)).logical_or(~valid).all())
+    cnt = valid.sum(-1)
+    assert bool((cnt == torch.clamp(nc, max=sh.K).view(1, 1, -1)).all())
+    d = idx[..., 1:] - idx[..., :-1]
+    assert bool(((d > 0) | ~valid[..., 1:]).all())

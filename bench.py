@@ -1,0 +1,509 @@
+#!/usr/bin/env python
+"""Benchmark of the HiLS attention forward path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl hils|reference] [--no-decode] [--no-cpu]
+
+One step = one HiLS prefill forward (landmark scoring + group top-K +
+gathered intra-chunk/window attention + chunk-softmax fusion) over the
+workload's whole synthetic input, through the C ABI (hils_prefill_select then
+hils_prefill_attend, exactly what hils_fwd_prefill runs), inputs resident in
+HBM. The default workload is the 32K prefill (B=1, Hq=32, Hkv=8, d=128,
+S=64, W=512, K=16, planted needles). The decode step of the 512K, batch-8
+workload is measured in the same run (as a CUDA graph) and reported under
+"decode". L2 is flushed (256 MiB write) before every timed step.
+
+Rank 0 prints one JSON line. Under torchrun each rank runs its own replica of
+the workload on its own GPU (the path shards by (batch, kv head) with no
+exchange), timed with CUDA events, max over ranks.
+
+--impl reference times the fp64 CPU oracle (the reference arm of this
+build) on a bounded sample of query positions per step.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = ("HiLS fwd prefill tokens/s & decode µs/token at 1 B200; "
+          "% of tensor/HBM roofline")
+WORKLOADS = {"prefill_32k": 2, "prefill_128k": 3, "prefill_512k": 5}
+DECODE_WORKLOAD = ("decode_512k_b8", 4)
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------ work counting
+def prefill_work(sh):
+    """Algorithmic work of one prefill forward (touched, not executed):
+    select FLOPs = sum_rows Hq * 2d|C_i|; attend FLOPs = sum_rows Hq *
+    4d(|I_i| S + i - w0 + 1); HBM bytes of the inputs read once and outputs
+    written once."""
+    i = np.arange(sh.N, dtype=np.int64)
+    lq = np.floor_divide(i - sh.W + 1, sh.S)
+    nc = np.maximum(lq, 0)
+    w0 = np.maximum(lq * sh.S, 0)
+    sel = np.minimum(nc, sh.K)
+    toks = sel * sh.S + (i - w0 + 1)
+    f_select = float(sh.B * sh.Hq * 2 * sh.d * nc.sum())
+    f_attend = float(sh.B * sh.Hq * 4 * sh.d * toks.sum())
+    return dict(select_flops=f_select, attend_flops=f_attend,
+                tokens=sh.B * sh.N)
+
+
+def decode_bytes(sh, cache_len):
+    """Touched HBM bytes of one decode step: k' and b' of every candidate,
+    K and V of the selected chunks and the window, Q, O, idx."""
+    tot = 0
+    esz = 2 if sh.dtype == "bf16" else 4
+    for L in cache_len:
+        i = L - 1
+        lq = (i - sh.W + 1) // sh.S
+        nc = max(lq, 0)
+        w0 = max(lq * sh.S, 0)
+        toks = min(nc, sh.K) * sh.S + (i - w0 + 1)
+        tot += nc * sh.Hkv * (sh.d * esz + 4)
+        tot += toks * sh.Hkv * 2 * sh.d * esz
+        tot += 2 * sh.Hq * sh.d * esz + sh.Hkv * sh.K * 4
+    return float(tot)
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,"
+         "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]),
+                                 power=float(f[3]), hw=f[5], hwt=f[6],
+                                 swt=f[7], pcap=f[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for k, n in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                         ("swt", "sw_thermal_slowdown"),
+                         ("pcap", "sw_power_cap")):
+                if r[k].lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["smax"] for r in rows),
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sustained=d.get("bf16_tflops_sustained",
+                                         d["bf16_tflops"]),
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0,
+                src="fallback")
+
+
+# -------------------------------------------------------------- oracle arm
+def oracle_sample(inp, budget_s, positions_per_batch=8, seed=0,
+                  max_batches=None):
+    """Time the fp64 oracle on random query positions of the workload until
+    `budget_s` seconds of work. Returns (tokens/s, positions, seconds,
+    threads)."""
+    import oracle
+    sh = inp["shape"]
+    rng = np.random.default_rng(seed)
+    bound = oracle.bind_prefill(inp)
+    done, t0 = 0, time.perf_counter()
+    nb = 0
+    while True:
+        pos = rng.integers(0, sh.N, size=positions_per_batch)
+        rows = np.array([[b, g, i] for b in range(sh.B)
+                         for g in range(sh.Hkv) for i in pos])
+        oracle.prefill_rows(inp, rows, bound=bound)
+        done += len(pos) * sh.B
+        nb += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or (max_batches and nb >= max_batches):
+            break
+    return done / el, done, el, oracle.max_threads()
+
+
+def host_inputs(inp):
+    import torch
+    out = {}
+    for k in ("Q", "K", "V", "Klm", "bias"):
+        t = inp[k].cpu()
+        out[k] = t.pin_memory() if torch.cuda.is_available() else t
+    return out
+
+
+def run_reference(args, sh, name):
+    """The CPU oracle as the reference arm, on this arm's workload."""
+    import synth
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    inp = synth.make_prefill(sh, seed=synth.seed_for(WORKLOADS[name]),
+                             device="cpu")
+    per_step = []
+    cnt = []
+    for s in range(args.warmup + args.steps):
+        v, n, el, thr = oracle_sample(inp, budget_s=0.0,
+                                      positions_per_batch=4, seed=s,
+                                      max_batches=1)
+        if s >= args.warmup:
+            per_step.append(el)
+            cnt.append(n)
+    tot = sum(per_step)
+    val = sum(cnt) / tot
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val,
+        "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * tot / len(per_step),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": workload_config(sh, name),
+        "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": thr,
+                         "kind": "oracle",
+                         "sample": f"4 random query positions (all heads) "
+                                   f"per step of the {name} workload"},
+        "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(sh, name):
+    return {"workload": name, "B": sh.B, "Hq": sh.Hq, "Hkv": sh.Hkv,
+            "d": sh.d, "N": sh.N, "S": sh.S, "W": sh.W, "K": sh.K,
+            "structure": sh.structure,
+            "l2": "flushed by a 256 MiB write before every timed step",
+            "parallelism": "one independent replica per GPU (shards by "
+                           "(batch, kv head), no collective)"}
+
+
+# ---------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill_32k",
+                    choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="hils", choices=["hils", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    import synth
+    cfg_id = WORKLOADS[args.workload]
+    sh = synth.PREFILL_CONFIGS[cfg_id]
+    if args.impl == "reference":
+        run_reference(args, sh, args.workload)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import chunk_sparse_long_landmark_b200 as hils
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks = measured_peaks()
+    inp = synth.make_prefill(sh, seed=synth.seed_for(cfg_id) + 17 * rank,
+                             device=dev)
+    work = prefill_work(sh)
+    B, Hq, Hkv, N, d, K = sh.B, sh.Hq, sh.Hkv, sh.N, sh.d, sh.K
+    O = torch.empty_like(inp["Q"])
+    idx = torch.empty(B, Hkv, N, K, dtype=torch.int32, device=dev)
+    sel = torch.empty(B, Hq, N, K, dtype=torch.float32, device=dev)
+    ws = torch.empty(hils.prefill_workspace_size(
+        inp["Q"], inp["K"], inp["V"], inp["Klm"], inp["bias"],
+        inp["head_map"], sh.S, sh.W, K, with_sel_score=True),
+        dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def call(stage):
+        hils.fwd_prefill(inp["Q"], inp["K"], inp["V"], inp["Klm"],
+                         inp["bias"], inp["head_map"], sh.S, sh.W, K,
+                         out=O, idx=idx, sel_score=sel, workspace=ws,
+                         stream=stream, stage=stage)
+
+    for _ in range(args.warmup):
+        call("select")
+        call("attend")
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+           for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    n0 = hils.launch_count()
+    with ClockSampler(local) as clk:
+        for s in range(args.steps):
+            flush.zero_()
+            evs[s][0].record(stream)
+            call("select")
+            evs[s][1].record(stream)
+            call("attend")
+            evs[s][2].record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    launches = hils.launch_count() - n0
+    t_sel = [e[0].elapsed_time(e[1]) for e in evs]
+    t_att = [e[1].elapsed_time(e[2]) for e in evs]
+    t_step = [a + b for a, b in zip(t_sel, t_att)]
+    tot_ms = max_over_ranks(sum(t_step))
+    ms_step = tot_ms / args.steps
+    value = world * work["tokens"] / (ms_step * 1e-3)
+
+    # dominant kernel roofline (tensor-bound contraction)
+    a_ms, s_ms = statistics.mean(t_att), statistics.mean(t_sel)
+    if a_ms >= s_ms:
+        dom, dom_ms, dom_flops = "attend", a_ms, work["attend_flops"]
+    else:
+        dom, dom_ms, dom_flops = "select", s_ms, work["select_flops"]
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    peak = peaks["bf16_sustained"] if args.steps * ms_step > 2000 else \
+        peaks["bf16"]
+    roof = {"bound": "tensor", "kernel": dom, "achieved": achieved,
+            "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_source": peaks["src"],
+            "algorithmic_flops_per_launch": dom_flops, "traffic": None}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(sh, args.workload),
+        "stages_ms": {"select": s_ms, "attend": a_ms},
+        "roofline": roof,
+        "gpu_launches": int(launches),
+        "clocks": clk.summary(),
+    }
+
+    # end to end through the C ABI with host buffers (pinned), per step:
+    # H2D of Q, K, V, Klm, bias; the call; D2H of O and idx
+    if not args.no_e2e:
+        host = host_inputs(inp)
+        Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+        Ih = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = Oh.numel() * Oh.element_size() + Ih.numel() * Ih.element_size()
+        dvs = {k: torch.empty_like(inp[k]) for k in host}
+
+        def e2e_step():
+            for k, t in host.items():
+                dvs[k].copy_(t, non_blocking=True)
+            hils.fwd_prefill(dvs["Q"], dvs["K"], dvs["V"], dvs["Klm"],
+                             dvs["bias"], inp["head_map"], sh.S, sh.W, K,
+                             out=O, idx=idx, sel_score=sel, workspace=ws,
+                             stream=stream)
+            Oh.copy_(O, non_blocking=True)
+            Ih.copy_(idx, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        ee = [(torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True))
+              for _ in range(max(3, args.steps // 4))]
+        for a, b in ee:
+            flush.zero_()
+            a.record(stream)
+            e2e_step()
+            b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ee)) / len(ee)
+        line["e2e"] = {"value": world * work["tokens"] / (e_ms * 1e-3),
+                       "unit": "tokens/s", "ms_per_step": e_ms,
+                       "h2d_bytes_per_step": int(h2d),
+                       "d2h_bytes_per_step": int(d2h)}
+        del host, dvs
+
+    del inp, O, idx, sel, ws
+    torch.cuda.empty_cache()
+
+    if not args.no_decode:
+        line["decode"] = bench_decode(args, dev, stream, flush, world,
+                                      max_over_ranks, barrier, rank, peaks)
+
+    if rank == 0 and world == 1 and not args.no_cpu:
+        cinp = synth.make_prefill(sh, seed=synth.seed_for(cfg_id),
+                                  device=dev)
+        v, n, el, thr = oracle_sample(cinp, budget_s=15.0)
+        line["cpu_baseline"] = {
+            "value": v, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+            "sample": f"{n} random query positions (all {Hq} heads) of the "
+                      f"{args.workload} workload, {el:.1f} s"}
+        del cinp
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def bench_decode(args, dev, stream, flush, world, max_over_ranks, barrier,
+                 rank, peaks):
+    import torch
+
+    import chunk_sparse_long_landmark_b200 as hils
+    import synth
+    name, cid = DECODE_WORKLOAD
+    sh = synth.DECODE_CONFIGS[cid]
+    inp = synth.make_decode(sh, seed=synth.seed_for(cid) + 17 * rank,
+                            device=dev)
+    O = torch.empty_like(inp["Q"])
+    idx = torch.empty(sh.B, sh.Hkv, sh.K, dtype=torch.int32, device=dev)
+    sel = torch.empty(sh.B, sh.Hq, sh.K, dtype=torch.float32, device=dev)
+    ws = torch.empty(hils.decode_workspace_size(
+        inp["Q"], inp["K"], inp["V"], inp["Klm"], inp["bias"],
+        inp["cache_len"], inp["head_map"], sh.S, sh.W, sh.K,
+        with_sel_score=True), dtype=torch.uint8, device=dev)
+    side = torch.cuda.Stream(dev)
+
+    def call(st, stage="both"):
+        hils.fwd_decode(inp["Q"], inp["K"], inp["V"], inp["Klm"],
+                        inp["bias"], inp["cache_len"], inp["head_map"], sh.S,
+                        sh.W, sh.K, out=O, idx=idx, sel_score=sel,
+                        workspace=ws, stream=st, stage=stage)
+
+    with torch.cuda.stream(side):
+        for _ in range(args.warmup):
+            call(side)
+    side.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        call(side)
+    torch.cuda.synchronize()
+    steps = max(args.steps, 20)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier()
+    evs = [(torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    cur = torch.cuda.current_stream(dev)
+    for a, b in evs:
+        flush.zero_()
+        a.record(cur)
+        g.replay()
+        b.record(cur)
+    torch.cuda.synchronize()
+    times = [a.elapsed_time(b) for a, b in evs]
+    ms = max_over_ranks(sum(times)) / steps
+    med = statistics.median(times)
+    # stage split (eager, separate events)
+    ss = []
+    for _ in range(5):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        flush.zero_()
+        e[0].record(cur)
+        call(cur, "select")
+        e[1].record(cur)
+        call(cur, "attend")
+        e[2].record(cur)
+        torch.cuda.synchronize()
+        ss.append((e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])))
+    cl = inp["cache_len"].cpu().tolist()
+    nbytes = decode_bytes(sh, cl)
+    ach = nbytes / (ms * 1e-3) / 1e9
+    del g
+    out = {
+        "workload": name, "value": ms * 1e3, "unit": "us/step",
+        "note": "one decode step = one new token for each of the B=8 "
+                "sequences (per-token latency of every sequence)",
+        "median_us": med * 1e3, "tokens_per_s": world * sh.B / (ms * 1e-3),
+        "stages_ms": {"select": statistics.mean(x[0] for x in ss),
+                      "attend": statistics.mean(x[1] for x in ss)},
+        "roofline": {"bound": "hbm", "kernel": "whole decode step (graph)",
+                     "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": ach / peaks["hbm"], "peak_source": peaks["src"],
+                     "algorithmic_bytes_per_step": nbytes, "traffic": None},
+        "config": {"B": sh.B, "Hq": sh.Hq, "Hkv": sh.Hkv, "d": sh.d,
+                   "L": sh.N, "S": sh.S, "W": sh.W, "K": sh.K,
+                   "l2": "flushed before every timed step"},
+    }
+    del inp, O, idx, sel, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+if __name__ == "__main__":
+    main()

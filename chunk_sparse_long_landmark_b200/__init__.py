@@ -18,6 +18,7 @@ __all__ = [
     "HilsError", "lib", "library_path", "symbols", "status_string",
     "fwd_prefill", "fwd_decode", "prefill_workspace_size",
     "decode_workspace_size", "PrefillArgs", "DecodeArgs", "STATUS",
+    "launch_count",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,6 +36,8 @@ F32, BF16 = 0, 1
 symbols = [
     "hils_status_string", "hils_version", "hils_prefill_workspace_size",
     "hils_decode_workspace_size", "hils_fwd_prefill", "hils_fwd_decode",
+    "hils_prefill_select", "hils_prefill_attend", "hils_decode_select",
+    "hils_decode_attend", "hils_launch_count",
 ]
 
 
@@ -87,9 +90,12 @@ def lib():
                 f = getattr(L, f"hils_{n}_workspace_size")
                 f.restype = ctypes.c_int
                 f.argtypes = [ctypes.POINTER(T), ctypes.POINTER(ctypes.c_size_t)]
-                f = getattr(L, f"hils_fwd_{n}")
-                f.restype = ctypes.c_int
-                f.argtypes = [ctypes.POINTER(T), ctypes.c_void_p]
+                for fn in (f"hils_fwd_{n}", f"hils_{n}_select",
+                           f"hils_{n}_attend"):
+                    f = getattr(L, fn)
+                    f.restype = ctypes.c_int
+                    f.argtypes = [ctypes.POINTER(T), ctypes.c_void_p]
+            L.hils_launch_count.restype = ctypes.c_uint64
             _lib = L
     return _lib
 
@@ -156,10 +162,23 @@ def prefill_workspace_size(Q, K, V, Klm, bias, head_map, S, W, topk,
     return int(n.value)
 
 
+def launch_count() -> int:
+    """Kernel launches libhils has enqueued in this process so far."""
+    return int(lib().hils_launch_count())
+
+
+_STAGE_FN = {"both": "hils_fwd_{}", "select": "hils_{}_select",
+             "attend": "hils_{}_attend"}
+
+
 def fwd_prefill(Q, K, V, Klm, bias, head_map, S, W, topk, Qs=None, out=None,
                 idx=None, sel_score=None, workspace=None, status=None,
-                stream=None):
+                stream=None, stage="both"):
     """HiLS prefill forward through hils_fwd_prefill. Returns (O, idx).
+
+    stage="select" / "attend" calls hils_prefill_select / _attend instead
+    (attend needs the idx and scores of a select call: pass sel_score, or the
+    same workspace, to both).
 
     Q/Qs [B,Hq,N,d], K/V [B,Hkv,N,d], Klm [B,Hkv,N//S,d] (same dtype),
     bias [B,Hkv,N//S] float32, head_map: Hq ints. Outputs are allocated with
@@ -179,9 +198,10 @@ def fwd_prefill(Q, K, V, Klm, bias, head_map, S, W, topk, Qs=None, out=None,
         workspace = torch.empty(n, dtype=torch.uint8, device=Q.device)
     a, hm = _prefill_struct(Q, K, V, Klm, bias, head_map, S, W, topk, Qs,
                             out, idx, sel_score, workspace, status)
-    rc = lib().hils_fwd_prefill(ctypes.byref(a), _stream_handle(stream))
+    fn = _STAGE_FN[stage].format("prefill")
+    rc = getattr(lib(), fn)(ctypes.byref(a), _stream_handle(stream))
     if rc:
-        raise HilsError(rc, "hils_fwd_prefill")
+        raise HilsError(rc, fn)
     return out, idx
 
 
@@ -215,7 +235,7 @@ def decode_workspace_size(Q, K, V, Klm, bias, cache_len, head_map, S, W,
 
 def fwd_decode(Q, K, V, Klm, bias, cache_len, head_map, S, W, topk, Qs=None,
                out=None, idx=None, sel_score=None, workspace=None,
-               status=None, stream=None):
+               status=None, stream=None, stage="both"):
     """HiLS decode step through hils_fwd_decode. Returns (O, idx).
 
     Q/Qs [B,Hq,d]; K/V caches [B,Hkv,Lmax,d]; Klm [B,Hkv,Lmax//S,d];
@@ -236,7 +256,8 @@ def fwd_decode(Q, K, V, Klm, bias, cache_len, head_map, S, W, topk, Qs=None,
         workspace = torch.empty(n, dtype=torch.uint8, device=Q.device)
     a, hm = _decode_struct(Q, K, V, Klm, bias, cache_len, head_map, S, W,
                            topk, Qs, out, idx, sel_score, workspace, status)
-    rc = lib().hils_fwd_decode(ctypes.byref(a), _stream_handle(stream))
+    fn = _STAGE_FN[stage].format("decode")
+    rc = getattr(lib(), fn)(ctypes.byref(a), _stream_handle(stream))
     if rc:
-        raise HilsError(rc, "hils_fwd_decode")
+        raise HilsError(rc, fn)
     return out, idx

@@ -10,7 +10,11 @@ namespace hils {
 bool fast_path_supported(const Problem &p);
 // Scratch bytes the fast kernels need inside the caller's workspace.
 size_t fast_workspace_bytes(const Problem &p);
-// Enqueue the fast kernels. `ws` is 256-byte aligned, `ws_bytes` as above.
-cudaError_t launch_fast(Problem &p, void *ws, size_t ws_bytes, cudaStream_t st);
+// Enqueue the fast kernels of one stage (each counts its own launches).
+// `ws` is 256-byte aligned, `ws_bytes` as above.
+cudaError_t launch_fast_select(Problem &p, void *ws, size_t ws_bytes,
+                               cudaStream_t st);
+cudaError_t launch_fast_attend(Problem &p, void *ws, size_t ws_bytes,
+                               cudaStream_t st);
 
 }  // namespace hils

@@ -150,20 +150,54 @@ void plan_workspace(const Problem &p, bool user_sel, Plan *pl) {
     pl->total = off > 0 ? off : kAlign;
 }
 
+enum Stage { kSelect = 1, kAttend = 2, kBoth = 3 };
+
 hils_status run(Problem &p, const Plan &pl, void *ws, size_t ws_bytes,
-                cudaStream_t st) {
+                cudaStream_t st, int stages) {
     if (ws_bytes < pl.total) return HILS_ERR_WORKSPACE_TOO_SMALL;
     if (!ws) return HILS_ERR_INVALID_ARG;
     char *base = (char *)ws;
     if (!p.sel) p.sel = (float *)(base + pl.sel_off);
-    cudaError_t e;
+    cudaError_t e = cudaSuccess;
     if (pl.path == 1) {
-        e = launch_fast(p, base + pl.fast_off, pl.fast_bytes, st);
+        if (stages & kSelect)
+            e = launch_fast_select(p, base + pl.fast_off, pl.fast_bytes, st);
+        if (e == cudaSuccess && (stages & kAttend))
+            e = launch_fast_attend(p, base + pl.fast_off, pl.fast_bytes, st);
     } else {
-        e = launch_simt_score(p, (float *)(base + pl.scr_off), pl.score_grid, st);
-        if (e == cudaSuccess) e = launch_simt_attend(p, st);
+        if (stages & kSelect) {
+            e = launch_simt_score(p, (float *)(base + pl.scr_off),
+                                  pl.score_grid, st);
+            count_launches(1);
+        }
+        if (e == cudaSuccess && (stages & kAttend)) {
+            e = launch_simt_attend(p, st);
+            count_launches(1);
+        }
     }
     return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
+}
+
+hils_status prefill_entry(const hils_prefill_args *args, void *stream,
+                          int stages) {
+    Problem p;
+    hils_status s = prefill_problem(args, &p, true);
+    if (s != HILS_OK) return s;
+    Plan pl;
+    plan_workspace(p, args->sel_score != nullptr, &pl);
+    return run(p, pl, args->workspace, args->workspace_bytes,
+               (cudaStream_t)stream, stages);
+}
+
+hils_status decode_entry(const hils_decode_args *args, void *stream,
+                         int stages) {
+    Problem p;
+    hils_status s = decode_problem(args, &p, true);
+    if (s != HILS_OK) return s;
+    Plan pl;
+    plan_workspace(p, args->sel_score != nullptr, &pl);
+    return run(p, pl, args->workspace, args->workspace_bytes,
+               (cudaStream_t)stream, stages);
 }
 
 }  // namespace
@@ -211,23 +245,29 @@ hils_status hils_decode_workspace_size(const hils_decode_args *args,
 }
 
 hils_status hils_fwd_prefill(const hils_prefill_args *args, void *stream) {
-    Problem p;
-    hils_status s = prefill_problem(args, &p, true);
-    if (s != HILS_OK) return s;
-    Plan pl;
-    plan_workspace(p, args->sel_score != nullptr, &pl);
-    return run(p, pl, args->workspace, args->workspace_bytes,
-               (cudaStream_t)stream);
+    return prefill_entry(args, stream, kBoth);
+}
+
+hils_status hils_prefill_select(const hils_prefill_args *args, void *stream) {
+    return prefill_entry(args, stream, kSelect);
+}
+
+hils_status hils_prefill_attend(const hils_prefill_args *args, void *stream) {
+    return prefill_entry(args, stream, kAttend);
 }
 
 hils_status hils_fwd_decode(const hils_decode_args *args, void *stream) {
-    Problem p;
-    hils_status s = decode_problem(args, &p, true);
-    if (s != HILS_OK) return s;
-    Plan pl;
-    plan_workspace(p, args->sel_score != nullptr, &pl);
-    return run(p, pl, args->workspace, args->workspace_bytes,
-               (cudaStream_t)stream);
+    return decode_entry(args, stream, kBoth);
 }
+
+hils_status hils_decode_select(const hils_decode_args *args, void *stream) {
+    return decode_entry(args, stream, kSelect);
+}
+
+hils_status hils_decode_attend(const hils_decode_args *args, void *stream) {
+    return decode_entry(args, stream, kAttend);
+}
+
+uint64_t hils_launch_count(void) { return launch_total(); }
 
 }  // extern "C"

@@ -61,6 +61,10 @@ __device__ __forceinline__ void report(int32_t *status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
 
+// Process-wide count of kernel launches enqueued by the library.
+void count_launches(int n);
+uint64_t launch_total();
+
 // Kernel launchers (defined in the .cu files).
 cudaError_t launch_simt_score(const Problem &p, float *scratch, int grid,
                               cudaStream_t st);

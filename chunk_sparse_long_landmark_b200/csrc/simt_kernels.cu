@@ -218,8 +218,10 @@ simt_attend_kernel(const Problem p) {
 
     // reference point: the largest selected chunk score (every fused chunk
     // weight exp(s - m_c)/z_c * exp(s^_c - M) is then <= 1)
+    // idx entries outside C_i (caller-supplied selections) are ignored
     float M = -INFINITY;
-    for (int k = 0; k < K; ++k) if (io[k] >= 0) M = fmaxf(M, so[k]);
+    for (int k = 0; k < K; ++k)
+        if (io[k] >= 0 && io[k] < nc) M = fmaxf(M, so[k]);
     float l = 0.f;
 
     auto logit = [&](int64_t j) {
@@ -232,7 +234,7 @@ simt_attend_kernel(const Problem p) {
     // selected chunks: intra-chunk softmax, weighted by Z^_c (Sec. 3)
     for (int k = 0; k < K; ++k) {
         const int c = io[k];
-        if (c < 0) continue;
+        if (c < 0 || c >= nc) continue;
         float mc = -INFINITY;
         for (int t = lane; t < S; t += 32) {
             float s = logit((int64_t)c * S + t);

@@ -162,6 +162,32 @@ hils_status hils_fwd_prefill(const hils_prefill_args *args, void *stream);
  */
 hils_status hils_fwd_decode(const hils_decode_args *args, void *stream);
 
+/*
+ * The two stages of hils_fwd_prefill / hils_fwd_decode, callable alone (same
+ * argument record, same stream rules). hils_fwd_* is exactly select followed
+ * by attend.
+ *
+ * *_select: chunk scoring, per-head normaliser, group top-K (Sec. 3, Sec. 4.1).
+ *   Writes idx and the selected chunks' scores (sel_score, or the workspace
+ *   when sel_score is NULL). Reads Q / Qs, Klm, bias; O is not touched.
+ * *_attend: intra-chunk softmax attention over the chunks listed in idx and
+ *   the aligned window, fused with the chunk-level softmax (Sec. 3, RQ2).
+ *   Reads Q, Kc, V, idx and the selected scores; writes O. With sel_score
+ *   NULL it must be given the same workspace as the select call. idx entries
+ *   that are negative or not in C_i are ignored; each listed chunk must
+ *   appear once, in ascending order.
+ */
+hils_status hils_prefill_select(const hils_prefill_args *args, void *stream);
+hils_status hils_prefill_attend(const hils_prefill_args *args, void *stream);
+hils_status hils_decode_select(const hils_decode_args *args, void *stream);
+hils_status hils_decode_attend(const hils_decode_args *args, void *stream);
+
+/*
+ * Number of kernel launches this library has enqueued in this process so far
+ * (all devices, all threads). A diagnostic for counting launches per call.
+ */
+uint64_t hils_launch_count(void);
+
 #ifdef __cplusplus
 }
 #endif

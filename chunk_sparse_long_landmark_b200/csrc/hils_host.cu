@@ -65,7 +65,8 @@ struct Plan {
     size_t scr_off = 0, scr_bytes = 0;      // SIMT scoring scratch
     size_t fast_off = 0, fast_bytes = 0;    // fast-path scratch
     int score_grid = 0;
-    int path = 0;                           // 0: SIMT, 1: fast kernels
+    bool fast_select = false;               // tensor-core selection kernels
+    bool fast_attend = false;               // tensor-core attention kernels
     size_t total = 0;
 };
 
@@ -137,12 +138,14 @@ void plan_workspace(const Problem &p, bool user_sel, Plan *pl) {
         pl->sel_bytes = sizeof(float) * (size_t)p.B * p.Hq * p.n_query * p.K;
         off = align_up(off + pl->sel_bytes);
     }
-    pl->path = fast_path_supported(p) ? 1 : 0;
-    if (pl->path == 1) {
+    pl->fast_attend = fast_path_supported(p);
+    pl->fast_select = pl->fast_attend && fast_select_supported(p);
+    if (pl->fast_attend || pl->fast_select) {
         pl->fast_off = off;
         pl->fast_bytes = fast_workspace_bytes(p);
         off = align_up(off + pl->fast_bytes);
-    } else {
+    }
+    if (!pl->fast_select) {
         plan_simt_scratch(p, pl);
         pl->scr_off = off;
         off = align_up(off + pl->scr_bytes);
@@ -159,18 +162,19 @@ hils_status run(Problem &p, const Plan &pl, void *ws, size_t ws_bytes,
     char *base = (char *)ws;
     if (!p.sel) p.sel = (float *)(base + pl.sel_off);
     cudaError_t e = cudaSuccess;
-    if (pl.path == 1) {
-        if (stages & kSelect)
+    if (stages & kSelect) {
+        if (pl.fast_select) {
             e = launch_fast_select(p, base + pl.fast_off, pl.fast_bytes, st);
-        if (e == cudaSuccess && (stages & kAttend))
-            e = launch_fast_attend(p, base + pl.fast_off, pl.fast_bytes, st);
-    } else {
-        if (stages & kSelect) {
+        } else {
             e = launch_simt_score(p, (float *)(base + pl.scr_off),
                                   pl.score_grid, st);
             count_launches(1);
         }
-        if (e == cudaSuccess && (stages & kAttend)) {
+    }
+    if (e == cudaSuccess && (stages & kAttend)) {
+        if (pl.fast_attend) {
+            e = launch_fast_attend(p, base + pl.fast_off, pl.fast_bytes, st);
+        } else {
             e = launch_simt_attend(p, st);
             count_launches(1);
         }

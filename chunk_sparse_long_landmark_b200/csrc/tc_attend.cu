@@ -1,0 +1,472 @@
+// tc_attend.cu -- HiLS prefill gather-attention on the sm_100a tensor cores.
+//
+// "Hierarchical Sparse Attention Done Right", Sec. 3 (hierarchical softmax,
+// RQ2 display) and Sec. 4.2 (M adjacent queries x G heads share one tile).
+//
+// One CTA owns 128 rows = the G query heads of one kv group x M = 128/G
+// adjacent queries (row r = head_slot * M + query_slot). It loads the union
+// of the M queries' selected chunks once and then every tile of the aligned
+// window the block touches, each tile S tokens of K and V brought in by TMA:
+//   S   = Q K^T      tcgen05.mma, 128 x S_TOK, f32 accumulator in TMEM
+//   P   = softmax    per row, in registers (chunk tiles: intra-chunk softmax
+//                    scaled by exp(s^_c - M0)/z_c, zero for rows that did not
+//                    select the chunk; window tiles: causal + window mask,
+//                    running reference max)
+//   O  += P V        tcgen05.mma, 128 x d, A = P (bf16, smem), f32 in TMEM
+// Warp roles: warp 0 TMA producer, warp 1 MMA issuer (and TMEM owner),
+// warps 2-5 softmax / epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// All waits are bounded (sm100::mbar_wait): a lost arrival ends the kernel
+// with HILS_ERR_DEVICE_TIMEOUT in the status word.
+#include <math.h>
+
+#include "hils_fast.cuh"
+#include "sm100.cuh"
+#include "tc_kernels.cuh"
+
+namespace hils {
+namespace {
+
+using namespace sm100;
+
+constexpr int kThreads = 192;
+constexpr int kRows = 128;
+constexpr int kStages = 2;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleLog2 = 8.0f;      // lazy O rescale threshold (log2)
+
+template <int S_TOK, int D>
+struct AttnLayout {
+    static constexpr int NP = (S_TOK == 64) ? 2 : 1;           // P buffers
+    static constexpr uint32_t Q_BYTES = kRows * D * 2;
+    static constexpr uint32_t KV_BYTES = S_TOK * D * 2;        // one of K or V
+    static constexpr uint32_t P_BYTES = kRows * S_TOK * 2;
+    static constexpr uint32_t OFF_Q = 0;
+    static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
+    static constexpr uint32_t OFF_V = OFF_K + kStages * KV_BYTES;
+    static constexpr uint32_t OFF_P = OFF_V + kStages * KV_BYTES;
+    static constexpr uint32_t OFF_SMALL = OFF_P + NP * P_BYTES;
+    static constexpr int TMEM_O = 0;                 // columns [0, D)
+    static constexpr int TMEM_S = D;                 // 2 buffers of S_TOK
+    static constexpr uint32_t TMEM_COLS =
+        (D + 2 * S_TOK) <= 256 ? 256u : 512u;
+};
+
+struct SmallState {
+    uint64_t q_full;
+    uint64_t kv_full[kStages];
+    uint64_t kv_empty[kStages];
+    uint64_t s_full[2];
+    uint64_t s_empty[2];
+    uint64_t p_full[2];
+    uint64_t p_empty[2];
+    uint64_t mma_done;
+    uint32_t tmem_base;
+    int abort;
+    int n_union;
+    int n_win_tiles;
+    int win_start;
+};
+
+template <int S_TOK, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
+                 const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV,
+                 const TcParams p) {
+    using L = AttnLayout<S_TOK, D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    SmallState &st = *reinterpret_cast<SmallState *>(smem + L::OFF_SMALL);
+    int *s_idx = reinterpret_cast<int *>(smem + L::OFF_SMALL + sizeof(SmallState));
+    int *s_union = s_idx + p.M * p.K;
+    uint32_t *s_bits = reinterpret_cast<uint32_t *>(s_union + p.ucap);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nqb = (p.N + p.M - 1) / p.M;
+    const int qb = blockIdx.x % nqb;
+    const int g = (blockIdx.x / nqb) % p.Hkv;
+    const int b = blockIdx.x / (nqb * p.Hkv);
+    const int i0 = qb * p.M;
+    const int i_last = min(i0 + p.M, p.N) - 1;
+    volatile int *abort = &st.abort;
+
+    // ---------------------------------------------------------- prologue
+    if (threadIdx.x == 0) {
+        mbar_init(&st.q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&st.kv_full[s], 1);
+            mbar_init(&st.kv_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&st.s_full[s], 1);
+            mbar_init(&st.s_empty[s], 128);
+            mbar_init(&st.p_full[s], 128);
+            mbar_init(&st.p_empty[s], 1);
+        }
+        mbar_init(&st.mma_done, 1);
+        st.abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(&st.tmem_base, L::TMEM_COLS);
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmQ);
+        prefetch_tmap(&tmK);
+        prefetch_tmap(&tmV);
+    }
+    // selected chunks of the block's queries -> smem; union bitmap
+    const int nwords = (p.nC + 31) >> 5;
+    for (int w = threadIdx.x; w < nwords; w += kThreads) s_bits[w] = 0u;
+    __syncthreads();
+    for (int e = threadIdx.x; e < p.M * p.K; e += kThreads) {
+        const int m = e / p.K, k = e % p.K;
+        const int i = i0 + m;
+        int c = -1;
+        if (i < p.N) {
+            int64_t w0, nc;
+            window_bounds(i, p.S, p.W, &w0, &nc);
+            c = p.idx[(((int64_t)b * p.Hkv + g) * p.N + i) * p.K + k];
+            if (c < 0 || c >= nc) c = -1;
+        }
+        s_idx[e] = c;
+        if (c >= 0) atomicOr(&s_bits[c >> 5], 1u << (c & 31));
+    }
+    __syncthreads();
+    if (warp == 0) {                       // ascending compaction of the union
+        int base = 0;
+        for (int w0i = 0; w0i < nwords; w0i += 32) {
+            const int w = w0i + lane;
+            uint32_t bits = w < nwords ? s_bits[w] : 0u;
+            const int cnt = __popc(bits);
+            int incl = cnt;
+            for (int o = 1; o < 32; o <<= 1) {
+                int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int pos = base + incl - cnt;
+            while (bits) {
+                const int bit = __ffs(bits) - 1;
+                bits &= bits - 1;
+                if (pos < p.ucap) s_union[pos] = w * 32 + bit;
+                ++pos;
+            }
+            base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            st.n_union = min(base, p.ucap);
+            int64_t w0, nc;
+            window_bounds(i0, p.S, p.W, &w0, &nc);
+            st.win_start = (int)w0;
+            st.n_win_tiles = (i_last - (int)w0) / S_TOK + 1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = st.tmem_base;
+    const int U = st.n_union;
+    const int T = U + st.n_win_tiles;
+    const int wstart = st.win_start;
+
+    if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            mbar_expect_tx(&st.q_full, L::Q_BYTES);
+            for (int hh = 0; hh < p.G; ++hh) {
+                const int h = p.group_heads[g * p.G + hh];
+                for (int dh = 0; dh < D / 64; ++dh)
+                    tma_load_4d(smem + L::OFF_Q + dh * (kRows * 128) +
+                                    hh * p.M * 128,
+                                &tmQ, &st.q_full, dh * 64, i0, h, b);
+            }
+            int issued = 0;
+            for (int t = 0; t < T; ++t) {
+                const int s = t % kStages;
+                if (t >= kStages &&
+                    !mbar_wait(&st.kv_empty[s], ((t / kStages) - 1) & 1, abort))
+                    break;
+                const int row = (t < U) ? s_union[t] * p.S
+                                        : wstart + (t - U) * S_TOK;
+                mbar_expect_tx(&st.kv_full[s], 2 * L::KV_BYTES);
+                for (int dh = 0; dh < D / 64; ++dh) {
+                    tma_load_4d(smem + L::OFF_K + s * L::KV_BYTES +
+                                    dh * (S_TOK * 128),
+                                &tmK, &st.kv_full[s], dh * 64, row, g, b);
+                    tma_load_4d(smem + L::OFF_V + s * L::KV_BYTES +
+                                    dh * (S_TOK * 128),
+                                &tmV, &st.kv_full[s], dh * 64, row, g, b);
+                }
+                issued = t + 1;
+            }
+            // on abort: let the copies already issued land before exiting
+            if (*abort) {
+                mbar_drain(&st.q_full, 0);
+                for (int t = (issued > kStages ? issued - kStages : 0);
+                     t < issued; ++t)
+                    mbar_drain(&st.kv_full[t % kStages], (t / kStages) & 1);
+            }
+        }
+    } else if (warp == 1) {
+        // ----------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_s = idesc_bf16(kRows, S_TOK, false);
+            constexpr uint32_t id_o = idesc_bf16(kRows, D, true);
+            const uint32_t sQ = smem_u32(smem + L::OFF_Q);
+            const uint32_t sK = smem_u32(smem + L::OFF_K);
+            const uint32_t sV = smem_u32(smem + L::OFF_V);
+            const uint32_t sP = smem_u32(smem + L::OFF_P);
+            bool ok = mbar_wait(&st.q_full, 0, abort);
+            tc_fence_after();
+            auto do_pv = [&](int u) -> bool {
+                const int pb = u % L::NP;
+                if (!mbar_wait(&st.p_full[pb], (u / L::NP) & 1, abort)) return false;
+                tc_fence_after();
+                const int s = u % kStages;
+#pragma unroll
+                for (int k = 0; k < S_TOK / 16; ++k) {
+                    const uint64_t ad = desc_sw128(
+                        sP + pb * L::P_BYTES + (k / 4) * (kRows * 128) + (k % 4) * 32,
+                        16, 1024);
+                    const uint64_t bd = desc_sw128(
+                        sV + s * L::KV_BYTES + k * 16 * 128, S_TOK * 128, 1024);
+                    mma_ss(tmem + L::TMEM_O, ad, bd, id_o, (u > 0 || k > 0) ? 1u : 0u);
+                }
+                mma_commit(&st.kv_empty[s]);
+                mma_commit(&st.p_empty[pb]);
+                return true;
+            };
+            for (int t = 0; ok && t < T; ++t) {
+                const int s = t % kStages;
+                const int sb = t & 1;
+                if (!mbar_wait(&st.kv_full[s], (t / kStages) & 1, abort)) { ok = false; break; }
+                if (t >= 2 && !mbar_wait(&st.s_empty[sb], ((t >> 1) - 1) & 1, abort)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint64_t ad = desc_sw128(
+                        sQ + (k / 4) * (kRows * 128) + (k % 4) * 32, 16, 1024);
+                    const uint64_t bd = desc_sw128(
+                        sK + s * L::KV_BYTES + (k / 4) * (S_TOK * 128) + (k % 4) * 32,
+                        16, 1024);
+                    mma_ss(tmem + L::TMEM_S + sb * S_TOK, ad, bd, id_s, k > 0 ? 1u : 0u);
+                }
+                mma_commit(&st.s_full[sb]);
+                if (t >= 1 && !do_pv(t - 1)) { ok = false; break; }
+            }
+            if (ok && T > 0) do_pv(T - 1);
+            // every MMA of this CTA has completed before TMEM is released
+            mma_commit(&st.mma_done);
+            mbar_drain(&st.mma_done, 0);
+        }
+    } else {
+        // -------------------------------------------- softmax / epilogue
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const int hh = r / p.M, m = r % p.M;
+        const int i = i0 + m;
+        const bool valid = (hh < p.G) && (i < p.N);
+        const int h = valid ? p.group_heads[g * p.G + hh] : 0;
+        int64_t w0 = 0, nc = 0;
+        if (valid) window_bounds(i, p.S, p.W, &w0, &nc);
+        const int *myidx = s_idx + m * p.K;
+        const float *mysel = p.sel + (((int64_t)b * p.Hq + h) * p.N + i) * p.K;
+        float M0 = -INFINITY;                            // natural-log units
+        if (valid)
+            for (int k = 0; k < p.K; ++k)
+                if (myidx[k] >= 0) M0 = fmaxf(M0, mysel[k]);
+        const float M0l2 = M0 * kLog2e;
+        float mref = M0l2;                               // log2 units
+        float l = 0.f;
+        int kp = 0;
+        const float sl2 = p.inv_sqrt_d * kLog2e;
+        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        uint8_t *sP = smem + L::OFF_P;
+        bool ok = true;
+
+        for (int t = 0; t < T; ++t) {
+            const int sb = t & 1;
+            // every lane takes the same branch around warp-collective
+            // tcgen05.ld / st, so wait outcomes are agreed across the warp
+            if (!__all_sync(0xffffffffu, mbar_wait(&st.s_full[sb], (t >> 1) & 1, abort))) { ok = false; break; }
+            tc_fence_after();
+            float x[S_TOK];
+#pragma unroll
+            for (int c0 = 0; c0 < S_TOK; c0 += 32) {
+                uint32_t rr[32];
+                tmem_ld32(trow + L::TMEM_S + sb * S_TOK + c0, rr);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) x[c0 + j] = __uint_as_float(rr[j]) * sl2;
+            }
+            tc_fence_before();
+            mbar_arrive(&st.s_empty[sb]);
+
+            if (t < U) {
+                const int c = s_union[t];
+                while (kp < p.K && (myidx[kp] < 0 || myidx[kp] < c)) ++kp;
+                const bool sel = valid && kp < p.K && myidx[kp] == c;
+                if (sel) {
+                    const float sh = mysel[kp] * kLog2e;
+                    ++kp;
+                    float mc = x[0];
+#pragma unroll
+                    for (int j = 1; j < S_TOK; ++j) mc = fmaxf(mc, x[j]);
+                    float z = 0.f;
+#pragma unroll
+                    for (int j = 0; j < S_TOK; ++j) { x[j] = fast_exp2(x[j] - mc); z += x[j]; }
+                    const float wc = fast_exp2(sh - M0l2);
+                    l += wc;
+                    const float f = wc / z;
+#pragma unroll
+                    for (int j = 0; j < S_TOK; ++j) x[j] *= f;
+                } else {
+#pragma unroll
+                    for (int j = 0; j < S_TOK; ++j) x[j] = 0.f;
+                }
+            } else {
+                const int j0 = wstart + (t - U) * S_TOK;
+                float mx = -INFINITY;
+#pragma unroll
+                for (int j = 0; j < S_TOK; ++j) {
+                    const int pos = j0 + j;
+                    const bool in = valid && pos >= w0 && pos <= i;
+                    x[j] = in ? x[j] : -INFINITY;
+                    mx = fmaxf(mx, x[j]);
+                }
+                const bool mine = mx > mref + kRescaleLog2;
+                if (__any_sync(0xffffffffu, mine)) {
+                    // raise the reference max of the rows that need it and
+                    // rescale their O once PV(t-1) is done (warp-wide: the
+                    // TMEM load / store are collective; other rows use 1)
+                    const float fac = !mine ? 1.f
+                                    : (mref == -INFINITY) ? 0.f : fast_exp2(mref - mx);
+                    if (t >= 1) {
+                        const int u = t - 1;
+                        if (!__all_sync(0xffffffffu, mbar_wait(&st.p_empty[u % L::NP], (u / L::NP) & 1, abort))) { ok = false; break; }
+                        tc_fence_after();
+#pragma unroll
+                        for (int c0 = 0; c0 < D; c0 += 32) {
+                            uint32_t rr[32];
+                            tmem_ld32(trow + L::TMEM_O + c0, rr);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 32; ++j)
+                                rr[j] = __float_as_uint(__uint_as_float(rr[j]) * fac);
+                            tmem_st32(trow + L::TMEM_O + c0, rr);
+                        }
+                        tmem_wait_st();
+                    }
+                    if (mine) { l *= fac; mref = mx; }
+                }
+                float es = 0.f;
+#pragma unroll
+                for (int j = 0; j < S_TOK; ++j) {
+                    x[j] = (x[j] == -INFINITY) ? 0.f : fast_exp2(x[j] - mref);
+                    es += x[j];
+                }
+                l += es;
+            }
+
+            // P -> smem (bf16, K-major, 128B swizzle), then hand to the MMA
+            const int pb = t % L::NP;
+            if (t >= L::NP) {
+                const int u = t - L::NP;
+                if (!__all_sync(0xffffffffu, mbar_wait(&st.p_empty[pb], (u / L::NP) & 1, abort))) { ok = false; break; }
+            }
+            uint8_t *prow = sP + pb * L::P_BYTES + r * 128;
+#pragma unroll
+            for (int half = 0; half < S_TOK / 64; ++half) {
+#pragma unroll
+                for (int uu = 0; uu < 8; ++uu) {
+                    const int j = half * 64 + uu * 8;
+                    uint4 v;
+                    v.x = pack_bf16(x[j + 0], x[j + 1]);
+                    v.y = pack_bf16(x[j + 2], x[j + 3]);
+                    v.z = pack_bf16(x[j + 4], x[j + 5]);
+                    v.w = pack_bf16(x[j + 6], x[j + 7]);
+                    *reinterpret_cast<uint4 *>(prow + half * (kRows * 128) +
+                                               ((uu ^ (r & 7)) << 4)) = v;
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(&st.p_full[pb]);
+        }
+
+        // final: O / l once the last PV is done
+        if (ok && T > 0) {
+            const int u = T - 1;
+            ok = __all_sync(0xffffffffu, mbar_wait(&st.p_empty[u % L::NP], (u / L::NP) & 1, abort));
+        }
+        if (ok) {
+            tc_fence_after();
+            const float inv = (l > 0.f) ? 1.f / l : 0.f;
+            __nv_bfloat16 *orow = reinterpret_cast<__nv_bfloat16 *>(p.O) +
+                                  (((int64_t)b * p.Hq + h) * p.N + i) * D;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t rr[32];
+                tmem_ld32(trow + L::TMEM_O + c0, rr);
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8) {
+                        uint4 v;
+                        v.x = pack_bf16(__uint_as_float(rr[j + 0]) * inv, __uint_as_float(rr[j + 1]) * inv);
+                        v.y = pack_bf16(__uint_as_float(rr[j + 2]) * inv, __uint_as_float(rr[j + 3]) * inv);
+                        v.z = pack_bf16(__uint_as_float(rr[j + 4]) * inv, __uint_as_float(rr[j + 5]) * inv);
+                        v.w = pack_bf16(__uint_as_float(rr[j + 6]) * inv, __uint_as_float(rr[j + 7]) * inv);
+                        *reinterpret_cast<uint4 *>(orow + c0 + j) = v;
+                    }
+                }
+            }
+        }
+    }
+
+    // ------------------------------------------------------------ teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::TMEM_COLS);
+    }
+    if (threadIdx.x == 0 && st.abort) report(p.status, HILS_ERR_DEVICE_TIMEOUT);
+}
+
+template <int S_TOK, int D>
+cudaError_t launch_attend_t(const TcParams &tp, const TcMaps &maps,
+                            cudaStream_t st) {
+    using L = AttnLayout<S_TOK, D>;
+    const size_t smem = tc_attend_smem_bytes(tp, S_TOK, D);
+    auto kern = tc_attend_kernel<S_TOK, D>;
+    cudaError_t e = cudaFuncSetAttribute(
+        kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int nqb = (tp.N + tp.M - 1) / tp.M;
+    const int64_t grid = (int64_t)tp.B * tp.Hkv * nqb;
+    if (grid <= 0) return cudaSuccess;
+    kern<<<(unsigned)grid, kThreads, smem, st>>>(maps.q, maps.k, maps.v, tp);
+    (void)sizeof(L);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t tc_attend_smem_bytes(const TcParams &tp, int s_tok, int d) {
+    const int np = (s_tok == 64) ? 2 : 1;
+    size_t big = (size_t)kRows * d * 2 + 2ull * kStages * s_tok * d * 2 +
+                 (size_t)np * kRows * s_tok * 2;
+    size_t small = sizeof(SmallState) + sizeof(int) * ((size_t)tp.M * tp.K + tp.ucap) +
+                   sizeof(uint32_t) * (((size_t)tp.nC + 31) / 32);
+    return 1024 + big + ((small + 15) / 16) * 16;
+}
+
+cudaError_t launch_tc_attend(const TcParams &tp, const TcMaps &maps,
+                             cudaStream_t st) {
+    if (tp.S == 64 && tp.d == 128) return launch_attend_t<64, 128>(tp, maps, st);
+    if (tp.S == 64 && tp.d == 64) return launch_attend_t<64, 64>(tp, maps, st);
+    if (tp.S == 128 && tp.d == 128) return launch_attend_t<128, 128>(tp, maps, st);
+    if (tp.S == 128 && tp.d == 64) return launch_attend_t<128, 64>(tp, maps, st);
+    return cudaErrorNotSupported;
+}
+
+}  // namespace hils

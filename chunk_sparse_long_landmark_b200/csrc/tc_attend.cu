@@ -104,7 +104,9 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
             mbar_init(&st.p_empty[s], 1);
         }
         mbar_init(&st.mma_done, 1);
-        st.abort = 0;
+        // a CTA that timed out already: the rest of the grid skips its work
+        st.abort = (p.status && *(volatile int32_t *)p.status ==
+                                    HILS_ERR_DEVICE_TIMEOUT) ? 1 : 0;
         fence_barrier_init();
     }
     if (warp == 1) tmem_alloc(&st.tmem_base, L::TMEM_COLS);
@@ -164,10 +166,12 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
     tc_fence_after();
     const uint32_t tmem = st.tmem_base;
     const int U = st.n_union;
-    const int T = U + st.n_win_tiles;
+    const int T = st.abort ? 0 : U + st.n_win_tiles;
     const int wstart = st.win_start;
 
-    if (warp == 0) {
+    if (T == 0) {
+        // skipped (see above): straight to teardown
+    } else if (warp == 0) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
             mbar_expect_tx(&st.q_full, L::Q_BYTES);
@@ -423,6 +427,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
     }
 
     // ------------------------------------------------------------ teardown
+    if (*abort && (threadIdx.x & 31) == 0) report(p.status, HILS_ERR_DEVICE_TIMEOUT);
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {

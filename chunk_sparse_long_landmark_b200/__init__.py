@@ -18,7 +18,7 @@ __all__ = [
     "HilsError", "lib", "library_path", "symbols", "status_string",
     "fwd_prefill", "fwd_decode", "prefill_workspace_size",
     "decode_workspace_size", "PrefillArgs", "DecodeArgs", "STATUS",
-    "launch_count",
+    "launch_count", "fwd_decode_noalloc",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -37,7 +37,7 @@ symbols = [
     "hils_status_string", "hils_version", "hils_prefill_workspace_size",
     "hils_decode_workspace_size", "hils_fwd_prefill", "hils_fwd_decode",
     "hils_prefill_select", "hils_prefill_attend", "hils_decode_select",
-    "hils_decode_attend", "hils_launch_count",
+    "hils_decode_attend", "hils_launch_count", "hils_fwd_decode_noalloc",
 ]
 
 
@@ -96,6 +96,9 @@ def lib():
                     f.restype = ctypes.c_int
                     f.argtypes = [ctypes.POINTER(T), ctypes.c_void_p]
             L.hils_launch_count.restype = ctypes.c_uint64
+            L.hils_fwd_decode_noalloc.restype = ctypes.c_int
+            L.hils_fwd_decode_noalloc.argtypes = [ctypes.POINTER(DecodeArgs),
+                                                  ctypes.c_void_p]
             _lib = L
     return _lib
 
@@ -260,4 +263,26 @@ def fwd_decode(Q, K, V, Klm, bias, cache_len, head_map, S, W, topk, Qs=None,
     rc = getattr(lib(), fn)(ctypes.byref(a), _stream_handle(stream))
     if rc:
         raise HilsError(rc, fn)
+    return out, idx
+
+
+def fwd_decode_noalloc(Q, K, V, Klm, bias, cache_len, head_map, S, W, topk,
+                       Qs=None, out=None, idx=None, sel_score=None,
+                       status=None, stream=None):
+    """Decode step through hils_fwd_decode_noalloc: no workspace is passed;
+    the library's fixed device scratch is used. Returns (O, idx). Outputs are
+    allocated with torch here only when not given."""
+    import torch
+    _dev(Q, K, V, Klm, bias, cache_len, Qs, out, idx, sel_score, status)
+    B, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    if out is None:
+        out = torch.empty_like(Q)
+    if idx is None:
+        idx = torch.empty(B, Hkv, topk, dtype=torch.int32, device=Q.device)
+    a, hm = _decode_struct(Q, K, V, Klm, bias, cache_len, head_map, S, W,
+                           topk, Qs, out, idx, sel_score, None, status)
+    rc = lib().hils_fwd_decode_noalloc(ctypes.byref(a), _stream_handle(stream))
+    if rc:
+        raise HilsError(rc, "hils_fwd_decode_noalloc")
     return out, idx

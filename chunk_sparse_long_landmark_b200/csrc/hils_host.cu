@@ -206,6 +206,14 @@ hils_status decode_entry(const hils_decode_args *args, void *stream,
 
 }  // namespace
 
+namespace hils {
+// Full argument check of a decode record (shapes and pointers), shared with
+// the allocation-free entry point.
+hils_status decode_problem_checked(const hils_decode_args *a, Problem *p) {
+    return decode_problem(a, p, true);
+}
+}  // namespace hils
+
 extern "C" {
 
 const char *hils_status_string(hils_status s) {

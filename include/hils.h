@@ -183,6 +183,30 @@ hils_status hils_decode_select(const hils_decode_args *args, void *stream);
 hils_status hils_decode_attend(const hils_decode_args *args, void *stream);
 
 /*
+ * hils_fwd_decode without a caller workspace (the paper has no counterpart:
+ * this is a deployment variant). For callers that cannot allocate device
+ * memory when they call: a serving loop whose memory is reserved up front, a
+ * latency-critical path that cannot afford cudaMalloc's implicit device
+ * synchronisation, or a host with no way to size and own a workspace.
+ *
+ * Same record and semantics as hils_fwd_decode; `workspace` and
+ * `workspace_bytes` are ignored. Scratch comes from one fixed 8 MiB device
+ * array inside the library (every GPU that loads the library holds it until
+ * exit). It runs the CUDA-core decode kernels. The library allocates
+ * nothing on this path.
+ *   - The first call on a device, with that device current, looks up the
+ *     array's device address (cudaGetSymbolAddress); make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array and the next call overwrites it; calls
+ *     whose executions overlap on the GPU (different streams, concurrent
+ *     graphs) race on it. Nothing in it needs to start at zero.
+ *   - A shape whose scratch exceeds the array (sel_score NULL adds B*Hq*K
+ *     floats; scoring needs (Hq/Hkv + 1) * floor((Lmax-W)/S) floats per
+ *     block) returns HILS_ERR_WORKSPACE_TOO_SMALL without enqueuing work.
+ */
+hils_status hils_fwd_decode_noalloc(const hils_decode_args *args, void *stream);
+
+/*
  * Number of kernel launches this library has enqueued in this process so far
  * (all devices, all threads). A diagnostic for counting launches per call.
  */

@@ -86,8 +86,12 @@ uint64_t launch_total() { return g_launches.load(); }
 bool fast_path_supported(const Problem &p) { return attend_supported(p); }
 
 bool fast_select_supported(const Problem &p) {
-    (void)p;
-    return false;
+    if (p.decode || p.dtype != HILS_BF16) return false;
+    if (!(p.d == 64 || p.d == 128)) return false;
+    if (128 % p.G != 0 || p.nC < 1) return false;
+    if (!encode_fn()) return false;
+    TcParams tp = tc_params(p);
+    return tc_score_smem_bytes(tp, p.d) <= 227 * 1024;
 }
 
 size_t fast_workspace_bytes(const Problem &p) {
@@ -97,8 +101,14 @@ size_t fast_workspace_bytes(const Problem &p) {
 
 cudaError_t launch_fast_select(Problem &p, void *ws, size_t ws_bytes,
                                cudaStream_t st) {
-    (void)p; (void)ws; (void)ws_bytes; (void)st;
-    return cudaErrorNotSupported;
+    (void)ws; (void)ws_bytes;
+    TcParams tp = tc_params(p);
+    TcMaps maps;
+    if (!make_map(&maps.lm, p.Klm, p.d, p.nC, p.Hkv, p.B, 128))
+        return cudaErrorInvalidValue;
+    cudaError_t e = launch_tc_score(tp, maps, p.Qs ? p.Qs : p.Q, st);
+    count_launches(1);
+    return e;
 }
 
 cudaError_t launch_fast_attend(Problem &p, void *ws, size_t ws_bytes,

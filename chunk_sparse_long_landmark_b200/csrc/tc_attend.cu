@@ -77,8 +77,11 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     SmallState &st = *reinterpret_cast<SmallState *>(smem + L::OFF_SMALL);
+    // selected chunks of the block's queries, [K][M]; their scores for every
+    // row, [K][128]; the chunk union; its bitmap
     int *s_idx = reinterpret_cast<int *>(smem + L::OFF_SMALL + sizeof(SmallState));
-    int *s_union = s_idx + p.M * p.K;
+    float *s_sel = reinterpret_cast<float *>(s_idx + p.M * p.K);
+    int *s_union = reinterpret_cast<int *>(s_sel + kRows * p.K);
     uint32_t *s_bits = reinterpret_cast<uint32_t *>(s_union + p.ucap);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -120,7 +123,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
     for (int w = threadIdx.x; w < nwords; w += kThreads) s_bits[w] = 0u;
     __syncthreads();
     for (int e = threadIdx.x; e < p.M * p.K; e += kThreads) {
-        const int m = e / p.K, k = e % p.K;
+        const int m = e / p.K, k = e % p.K;      // consecutive e: one row's list
         const int i = i0 + m;
         int c = -1;
         if (i < p.N) {
@@ -129,8 +132,19 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
             c = p.idx[(((int64_t)b * p.Hkv + g) * p.N + i) * p.K + k];
             if (c < 0 || c >= nc) c = -1;
         }
-        s_idx[e] = c;
+        s_idx[k * p.M + m] = c;
         if (c >= 0) atomicOr(&s_bits[c >> 5], 1u << (c & 31));
+    }
+    for (int e = threadIdx.x; e < kRows * p.K; e += kThreads) {
+        const int r = e / p.K, k = e % p.K;
+        const int hh = r / p.M, m = r % p.M;
+        const int i = i0 + m;
+        float v = -INFINITY;
+        if (i < p.N && hh < p.G) {
+            const int h = p.group_heads[g * p.G + hh];
+            v = p.sel[(((int64_t)b * p.Hq + h) * p.N + i) * p.K + k];
+        }
+        s_sel[k * kRows + r] = v;
     }
     __syncthreads();
     if (warp == 0) {                       // ascending compaction of the union
@@ -271,12 +285,13 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
         const int h = valid ? p.group_heads[g * p.G + hh] : 0;
         int64_t w0 = 0, nc = 0;
         if (valid) window_bounds(i, p.S, p.W, &w0, &nc);
-        const int *myidx = s_idx + m * p.K;
-        const float *mysel = p.sel + (((int64_t)b * p.Hq + h) * p.N + i) * p.K;
+        const int *myidx = s_idx + m;                    // stride M
+        const float *mysel = s_sel + r;                  // stride 128
+        const int M_ = p.M;
         float M0 = -INFINITY;                            // natural-log units
         if (valid)
             for (int k = 0; k < p.K; ++k)
-                if (myidx[k] >= 0) M0 = fmaxf(M0, mysel[k]);
+                if (myidx[k * M_] >= 0) M0 = fmaxf(M0, mysel[k * kRows]);
         const float M0l2 = M0 * kLog2e;
         float mref = M0l2;                               // log2 units
         float l = 0.f;
@@ -306,10 +321,11 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
 
             if (t < U) {
                 const int c = s_union[t];
-                while (kp < p.K && (myidx[kp] < 0 || myidx[kp] < c)) ++kp;
-                const bool sel = valid && kp < p.K && myidx[kp] == c;
+                int ck = kp < p.K ? myidx[kp * M_] : 0x7fffffff;
+                while (kp < p.K && ck < c) { ++kp; ck = kp < p.K ? myidx[kp * M_] : 0x7fffffff; }
+                const bool sel = valid && kp < p.K && ck == c;
                 if (sel) {
-                    const float sh = mysel[kp] * kLog2e;
+                    const float sh = mysel[kp * kRows] * kLog2e;
                     ++kp;
                     float mc = x[0];
 #pragma unroll
@@ -461,6 +477,7 @@ size_t tc_attend_smem_bytes(const TcParams &tp, int s_tok, int d) {
     size_t big = (size_t)kRows * d * 2 + 2ull * kStages * s_tok * d * 2 +
                  (size_t)np * kRows * s_tok * 2;
     size_t small = sizeof(SmallState) + sizeof(int) * ((size_t)tp.M * tp.K + tp.ucap) +
+                   sizeof(float) * (size_t)kRows * tp.K +
                    sizeof(uint32_t) * (((size_t)tp.nC + 31) / 32);
     return 1024 + big + ((small + 15) / 16) * 16;
 }

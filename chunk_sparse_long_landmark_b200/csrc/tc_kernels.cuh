@@ -29,6 +29,9 @@ struct TcMaps {
     CUtensorMap lm; // Klm [B,Hkv,nC,d]: box {64, 128, 1, 1}
 };
 
+size_t tc_score_smem_bytes(const TcParams &tp, int d);
+cudaError_t launch_tc_score(const TcParams &tp, const TcMaps &maps,
+                            const void *qhat, cudaStream_t st);
 size_t tc_attend_smem_bytes(const TcParams &tp, int s_tok, int d);
 cudaError_t launch_tc_attend(const TcParams &tp, const TcMaps &maps,
                              cudaStream_t st);

@@ -1,0 +1,814 @@
+// decode_fast.cu -- HiLS decode step, HBM-bound kernels for sm_100a.
+//
+// "Hierarchical Sparse Attention Done Right", Sec. 3 (surrogate score, top-K,
+// hierarchical softmax) and Sec. 4.1 (GQA group selection), for one query
+// per sequence at i = cache_len-1 (the pages' decode setting, Sec. 7.1).
+//
+// The step reads every candidate landmark key once (the O(N/S) routing
+// scan) and the selected chunks + window of the caches once:
+//   dec_score   split over chunk ranges: 64-chunk landmark tiles by TMA,
+//               s^ for the G heads of the group (mma.sync m16n8k16 used as a
+//               dot-product engine: 16 chunks x 8 head slots x 16 dims),
+//               raw s^ -> workspace, per-split (max, sum-exp) per head.
+//   dec_select  one CTA per (b, kv head): merge the log-sum-exp partials,
+//               group score a_c = max_h (s^_hc - LSE_h), exact top-K by a
+//               4-round radix select (ties to the lower chunk), idx
+//               ascending, s^ of the selected chunks.
+//   dec_attend  one CTA per (b, kv head, selected chunk or window tile):
+//               K/V tile by TMA, QK^T and PV with mma.sync, intra-chunk
+//               softmax scaled by exp(s^_c) (chunk tiles) or plain masked
+//               softmax (window tiles) -> partial (m, l, o); the CTA that
+//               arrives last for its (b, kv head) combines the partials in
+//               tile order (deterministic) and writes O.
+#include <math.h>
+
+#include "hils_fast.cuh"
+#include "sm100.cuh"
+#include "tc_kernels.cuh"
+
+namespace hils {
+namespace {
+
+using namespace sm100;
+
+constexpr int kScoreWarps = 4;
+constexpr int kTileChunks = 64;                 // chunks per landmark tile
+constexpr int kScoreStages = 4;
+constexpr int kSelThreads = 1024;
+constexpr int kAttThreads = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct DecParams {
+    const void *Q, *Qs;
+    const float *bias;
+    const int32_t *cache_len;
+    void *O;
+    int32_t *idx;
+    float *sel;
+    int32_t *status;
+    float *ws_s;        // [B, Hkv, G, ncs] raw s^
+    float *ws_p;        // [B, Hkv, nsplit, G, 2] (max, sum exp(s^ - max))
+    float *ws_o;        // [B, Hkv, ntile, G, d] partial outputs
+    float *ws_ml;       // [B, Hkv, ntile, G, 2] partial (m, l)
+    int32_t *ws_cnt;    // [B, Hkv] arrival tickets
+    int B, Hq, Hkv, G, d, S, W, K, Lmax, nC;
+    int ncs;            // chunk stride of ws_s (max candidates of any row)
+    int nsplit;         // landmark splits per (b, g)
+    int cps;            // chunks per split (multiple of kTileChunks)
+    int ntile;          // attention tiles per (b, g): K + window tiles
+    float inv_sqrt_d;
+    int16_t group_heads[kMaxHeads];
+};
+
+__device__ __forceinline__ void mma_bf16(float *c, const uint32_t *a,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t *r) {
+    asm volatile("ldmatrix.sync.aligned.x4.m8n8.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t *r) {
+    asm volatile("ldmatrix.sync.aligned.x4.trans.m8n8.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map,
+                                            uint64_t *bar, int c0, int c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile"
+        ".mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        :: "r"(smem_u32(dst)), "l"((uint64_t)map), "r"(c0), "r"(c1),
+           "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Byte offset of 16-byte unit u of row r in a TMA 128B-swizzled tile whose
+// rows are 128 bytes (one 64-column half of a d=128 row).
+__device__ __forceinline__ uint32_t swz(int r, int u) {
+    return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ bool seq_ok(const DecParams &p, int b, int64_t *i,
+                                       int64_t *w0, int64_t *nc) {
+    const int L = p.cache_len[b];
+    if (L < 1 || L > p.Lmax) return false;
+    *i = L - 1;
+    window_bounds(*i, p.S, p.W, w0, nc);
+    return true;
+}
+
+// --------------------------------------------------------------- dec_score
+template <int D>
+__global__ void __launch_bounds__(kScoreWarps * 32)
+dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
+    constexpr int HALVES = D / 64;
+    constexpr uint32_t STAGE = kTileChunks * D * 2;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    __shared__ uint64_t full[kScoreStages];
+    __shared__ float red_m[kScoreWarps][8], red_s[kScoreWarps][8];
+
+    const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gi = lane >> 2, t = lane & 3;
+    const int G = p.G;
+    const int bg = b * p.Hkv + g;
+    if (split == 0 && threadIdx.x == 0) p.ws_cnt[bg] = 0;   // tickets of dec_attend
+    int64_t i, w0, nc;
+    const bool ok = seq_ok(p, b, &i, &w0, &nc);
+    if (!ok) {
+        if (split == 0 && threadIdx.x == 0) report(p.status, HILS_ERR_DEVICE_BAD_LENGTH);
+        return;
+    }
+    const int c_begin = split * p.cps;
+    const int c_end = (int)min((int64_t)c_begin + p.cps, nc);
+    const int ntiles = c_end > c_begin ? (c_end - c_begin + kTileChunks - 1) / kTileChunks : 0;
+
+    // scoring query as the B operand: column n = head slot gi (< G), rows = dims
+    const void *qb = p.Qs ? p.Qs : p.Q;
+    uint32_t bq[D / 16][2];
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+        bq[ks][0] = bq[ks][1] = 0u;
+        if (gi < G) {
+            const int h = p.group_heads[g * G + gi];
+            const uint32_t *q = reinterpret_cast<const uint32_t *>(
+                reinterpret_cast<const __nv_bfloat16 *>(qb) + ((int64_t)b * p.Hq + h) * D);
+            bq[ks][0] = q[(ks * 16 + 2 * t) >> 1];
+            bq[ks][1] = q[(ks * 16 + 8 + 2 * t) >> 1];
+        }
+    }
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kScoreStages; ++s) mbar_init(&full[s], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    const int64_t row0 = (int64_t)bg * p.nC + c_begin;
+    if (threadIdx.x == 0) {
+        for (int tt = 0; tt < min(ntiles, kScoreStages); ++tt) {
+            mbar_expect_tx(&full[tt], STAGE);
+            for (int hf = 0; hf < HALVES; ++hf)
+                tma_load_2d(smem + tt * STAGE + hf * (kTileChunks * 128), &tmL,
+                            &full[tt], hf * 64, (int)(row0 + tt * kTileChunks));
+        }
+    }
+    // per lane: heads 2t, 2t+1 (when < G); running max / sum in log2 units
+    float mx[2] = {-INFINITY, -INFINITY}, sm[2] = {0.f, 0.f};
+    const float sl2 = p.inv_sqrt_d * kLog2e;
+    const float *bias = p.bias + (int64_t)bg * p.nC;
+    float *outs = p.ws_s + (int64_t)bg * G * p.ncs;
+    volatile int dummy_abort = 0;
+    for (int tt = 0; tt < ntiles; ++tt) {
+        const int s = tt % kScoreStages;
+        mbar_wait(&full[s], (tt / kScoreStages) & 1, &dummy_abort);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t base = smem_u32(smem + s * STAGE);
+        const int r = warp * 16 + (lane & 15);
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const int hf = ks / 4, u = (ks % 4) * 2 + (lane >> 4);
+            uint32_t a[4];
+            ldsm_x4(base + hf * (kTileChunks * 128) + swz(r, u), a);
+            mma_bf16(acc, a, bq[ks][0], bq[ks][1]);
+        }
+        __syncthreads();                         // stage s fully read
+        if (threadIdx.x == 0 && tt + kScoreStages < ntiles) {
+            const int tn = tt + kScoreStages;
+            mbar_expect_tx(&full[s], STAGE);
+            for (int hf = 0; hf < HALVES; ++hf)
+                tma_load_2d(smem + s * STAGE + hf * (kTileChunks * 128), &tmL,
+                            &full[s], hf * 64, (int)(row0 + tn * kTileChunks));
+        }
+        // acc: chunks (gi, gi+8) of this warp's 16, heads (2t, 2t+1)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int hh = 2 * t + (q & 1);
+            const int c = c_begin + tt * kTileChunks + warp * 16 + gi + (q >> 1) * 8;
+            if (hh < G && c < c_end) {
+                const float shat = fmaf(acc[q], p.inv_sqrt_d, bias[c]);
+                outs[(int64_t)hh * p.ncs + c] = shat;
+                const float x = shat * kLog2e;
+                const int k = q & 1;
+                if (x > mx[k]) { sm[k] = sm[k] * fast_exp2(mx[k] - x) + 1.f; mx[k] = x; }
+                else sm[k] += fast_exp2(x - mx[k]);
+            }
+        }
+    }
+    (void)sl2;
+    if (dummy_abort) {                           // a tile never arrived
+        if (threadIdx.x == 0) {
+            report(p.status, HILS_ERR_DEVICE_TIMEOUT);
+            for (int tt = max(0, ntiles - kScoreStages); tt < ntiles; ++tt)
+                mbar_drain(&full[tt % kScoreStages], (tt / kScoreStages) & 1);
+        }
+        __syncthreads();
+        return;
+    }
+    // reduce (max, sum) over the 8 chunk lanes (gi) then over warps
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        for (int o = 4; o < 32; o <<= 1) {
+            const float om = __shfl_xor_sync(0xffffffffu, mx[k], o);
+            const float os = __shfl_xor_sync(0xffffffffu, sm[k], o);
+            const float mn = fmaxf(mx[k], om);
+            sm[k] = (mn == -INFINITY) ? 0.f
+                    : sm[k] * fast_exp2(mx[k] - mn) + os * fast_exp2(om - mn);
+            mx[k] = mn;
+        }
+    }
+    if (gi == 0) {
+        red_m[warp][2 * t] = mx[0]; red_s[warp][2 * t] = sm[0];
+        red_m[warp][2 * t + 1] = mx[1]; red_s[warp][2 * t + 1] = sm[1];
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
+        const int hh = threadIdx.x;
+        float m = -INFINITY, s2 = 0.f;
+        for (int w = 0; w < kScoreWarps; ++w) {
+            const float om = red_m[w][hh], os = red_s[w][hh];
+            const float mn = fmaxf(m, om);
+            s2 = (mn == -INFINITY) ? 0.f : s2 * fast_exp2(m - mn) + os * fast_exp2(om - mn);
+            m = mn;
+        }
+        float *pp = p.ws_p + (((int64_t)bg * p.nsplit + split) * G + hh) * 2;
+        pp[0] = m;          // log2 units
+        pp[1] = s2;
+    }
+}
+
+// -------------------------------------------------------------- dec_select
+__device__ __forceinline__ uint32_t order_key(float f) {
+    const uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// exclusive prefix over the block (kSelThreads threads) of v; returns it and
+// writes the block total to *total.
+__device__ int block_excl_scan(int v, int *scratch, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) scratch[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = scratch[lane];
+        int xi = w;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, xi, o);
+            if (lane >= o) xi += y;
+        }
+        scratch[lane] = xi - w;                  // exclusive warp offsets
+        if (lane == 31) scratch[32] = xi;
+    }
+    __syncthreads();
+    const int r = scratch[warp] + x - v;
+    *total = scratch[32];
+    __syncthreads();
+    return r;
+}
+
+constexpr int kSelPer = 16;                      // chunks per thread (<= 16384)
+
+__global__ void __launch_bounds__(kSelThreads)
+dec_select_kernel(const DecParams p) {
+    __shared__ float lse[HILS_MAX_GROUP];
+    __shared__ int hist[256];
+    __shared__ int scan_scr[33];
+    __shared__ int sh_digit, sh_need;
+    const int g = blockIdx.x, b = blockIdx.y;
+    const int bg = b * p.Hkv + g;
+    const int G = p.G, K = p.K;
+    int64_t i, w0, nc64;
+    if (!seq_ok(p, b, &i, &w0, &nc64)) return;
+    const int nc = (int)nc64;
+    const float *ss = p.ws_s + (int64_t)bg * G * p.ncs;
+
+    if (threadIdx.x < G) {                       // merge the split partials
+        const int hh = threadIdx.x;
+        float m = -INFINITY, s2 = 0.f;
+        const int nsp = (nc + p.cps - 1) / p.cps;
+        for (int sp = 0; sp < nsp; ++sp) {
+            const float *pp = p.ws_p + (((int64_t)bg * p.nsplit + sp) * G + hh) * 2;
+            const float om = pp[0], os = pp[1];
+            const float mn = fmaxf(m, om);
+            s2 = (mn == -INFINITY) ? 0.f : s2 * exp2f(m - mn) + os * exp2f(om - mn);
+            m = mn;
+        }
+        lse[hh] = (m == -INFINITY) ? 0.f : (m + log2f(s2)) / kLog2e;   // natural
+    }
+    __syncthreads();
+
+    // group scores of this thread's contiguous chunks c = tid * per + q
+    const int per = (nc + kSelThreads - 1) / kSelThreads;   // <= kSelPer
+    const int cbeg = threadIdx.x * per;
+    uint32_t key[kSelPer];
+#pragma unroll
+    for (int q = 0; q < kSelPer; ++q) {
+        const int c = cbeg + q;
+        key[q] = 0u;                             // below every real key
+        if (q < per && c < nc) {
+            float a = -INFINITY;
+            for (int hh = 0; hh < G; ++hh)
+                a = fmaxf(a, ss[(int64_t)hh * p.ncs + c] - lse[hh]);
+            key[q] = order_key(a);
+        }
+    }
+    const int nsel = min(nc, K);
+    uint32_t thr = 0u;                           // selected: key > thr, or == thr and early
+    int need_eq = 0;
+    if (nc > K) {
+        // radix select of the K-th largest key, 8 bits per round
+        uint32_t prefix = 0u, pmask = 0u;
+        int need = K;                            // still to take among matching keys
+        for (int shift = 24; shift >= 0; shift -= 8) {
+            for (int x = threadIdx.x; x < 256; x += kSelThreads) hist[x] = 0;
+            __syncthreads();
+#pragma unroll
+            for (int q = 0; q < kSelPer; ++q) {
+                const int c = cbeg + q;
+                if (q < per && c < nc && (key[q] & pmask) == prefix)
+                    atomicAdd(&hist[(key[q] >> shift) & 255], 1);
+            }
+            __syncthreads();
+            if (threadIdx.x < 32) {              // digit holding the need-th largest
+                const int lane = threadIdx.x;
+                int cnt[8], sum = 0;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) { cnt[k] = hist[255 - (lane * 8 + k)]; sum += cnt[k]; }
+                int incl = sum;                  // inclusive count from the top
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                int above = incl - sum;          // keys in higher digits of lower lanes
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    if (above < need && above + cnt[k] >= need) {
+                        sh_digit = 255 - (lane * 8 + k);
+                        sh_need = need - above;
+                    }
+                    above += cnt[k];
+                }
+            }
+            __syncthreads();
+            const int dg = sh_digit;
+            need = sh_need;
+            prefix |= (uint32_t)dg << shift;
+            pmask |= 255u << shift;
+            __syncthreads();
+        }
+        thr = prefix;                            // exact K-th largest key
+        need_eq = need;                          // how many keys equal to thr to take
+    }
+
+    // selected: key > thr, or key == thr among the first need_eq such chunks
+    // (chunk order = thread order, then q); positions in ascending chunk order
+    int n_eq = 0;
+#pragma unroll
+    for (int q = 0; q < kSelPer; ++q)
+        if (q < per && cbeg + q < nc && nc > K && key[q] == thr) ++n_eq;
+    int tot;
+    int rank_eq = block_excl_scan(n_eq, scan_scr, &tot);
+    uint32_t selbits = 0u;
+    int n_sel = 0;
+#pragma unroll
+    for (int q = 0; q < kSelPer; ++q) {
+        const int c = cbeg + q;
+        bool sc = false;
+        if (q < per && c < nc) {
+            if (nc <= K) sc = true;
+            else if (key[q] > thr) sc = true;
+            else if (key[q] == thr) { sc = rank_eq < need_eq; ++rank_eq; }
+        }
+        if (sc) { selbits |= 1u << q; ++n_sel; }
+    }
+    int pos = block_excl_scan(n_sel, scan_scr, &tot);
+    while (selbits) {
+        const int q = __ffs(selbits) - 1;
+        selbits &= selbits - 1;
+        const int c = cbeg + q;
+        if (pos < K) {
+            p.idx[(int64_t)bg * K + pos] = c;
+            for (int hh = 0; hh < G; ++hh) {
+                const int h = p.group_heads[g * G + hh];
+                p.sel[((int64_t)b * p.Hq + h) * K + pos] = ss[(int64_t)hh * p.ncs + c];
+            }
+        }
+        ++pos;
+    }
+    for (int k = nsel + threadIdx.x; k < K; k += kSelThreads) {
+        p.idx[(int64_t)bg * K + k] = -1;
+        for (int hh = 0; hh < G; ++hh) {
+            const int h = p.group_heads[g * G + hh];
+            p.sel[((int64_t)b * p.Hq + h) * K + k] = __int_as_float(0x7fc00000);
+        }
+    }
+}
+
+// -------------------------------------------------------------- dec_attend
+// One CTA = (b, kv head, group of kAttPer consecutive tiles of that (b, g)'s
+// tile list: the selected chunks in idx order, then the window tiles). The
+// CTA streams its tiles through a double-buffered TMA pipeline and merges
+// them online per head: running reference max M, O accumulated in the MMA
+// registers (rescaled when M rises), l in registers.
+constexpr int kAttPer = 6;                       // tiles per CTA
+
+template <int S_TOK, int D>
+__global__ void __launch_bounds__(kAttThreads)
+dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const DecParams p) {
+    constexpr int HALVES = D / 64;
+    constexpr uint32_t TB = S_TOK * D * 2;       // one of K or V
+    constexpr int TOK_W = S_TOK / 4;             // tokens per warp (16 or 32)
+    constexpr int NT = TOK_W / 8;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    __shared__ uint64_t bar[2];
+    __shared__ float red[4][8];
+    __shared__ int last;
+    float *ored = reinterpret_cast<float *>(smem + 4 * TB);     // [4][8][D]
+
+    const int grp = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int bg = b * p.Hkv + g;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int gi = lane >> 2, t = lane & 3;
+    const int G = p.G;
+    int64_t i = 0, w0 = 0, nc = 0;
+    const bool ok = seq_ok(p, b, &i, &w0, &nc);
+    int nsel = 0;
+    if (ok)
+        for (int k = 0; k < p.K; ++k) nsel += (p.idx[(int64_t)bg * p.K + k] >= 0) ? 1 : 0;
+    const int nwin = ok ? (int)((i - w0 + 1 + S_TOK - 1) / S_TOK) : 0;
+    const int ntot = nsel + nwin;
+    const int tb = grp * kAttPer;
+    const int te = min(tb + kAttPer, ntot);
+    const int nmine = te > tb ? te - tb : 0;
+    auto tile_j0 = [&](int tau) -> int64_t {
+        return tau < nsel ? (int64_t)p.idx[(int64_t)bg * p.K + tau] * p.S
+                          : w0 + (int64_t)(tau - nsel) * S_TOK;
+    };
+    volatile int dummy_abort = 0;
+    bool arrived_all = true;
+
+    if (nmine > 0) {
+        if (threadIdx.x == 0) {
+            mbar_init(&bar[0], 1);
+            mbar_init(&bar[1], 1);
+            fence_barrier_init();
+        }
+        __syncthreads();
+        auto issue = [&](int k) {                // tile tb + k into buffer k & 1
+            const int64_t row = (int64_t)bg * p.Lmax + tile_j0(tb + k);
+            uint8_t *dst = smem + (k & 1) * 2 * TB;
+            mbar_expect_tx(&bar[k & 1], 2 * TB);
+            for (int hf = 0; hf < HALVES; ++hf) {
+                tma_load_2d(dst + hf * (S_TOK * 128), &tmK, &bar[k & 1], hf * 64, (int)row);
+                tma_load_2d(dst + TB + hf * (S_TOK * 128), &tmV, &bar[k & 1], hf * 64, (int)row);
+            }
+        };
+        if (threadIdx.x == 0) {
+            issue(0);
+            if (nmine > 1) issue(1);
+        }
+        // Q as the A operand: row = head slot gi (< G), cols = dims
+        uint32_t aq[D / 16][4];
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            aq[ks][0] = aq[ks][1] = aq[ks][2] = aq[ks][3] = 0u;
+            if (gi < G) {
+                const int h = p.group_heads[g * G + gi];
+                const uint32_t *q = reinterpret_cast<const uint32_t *>(
+                    reinterpret_cast<const __nv_bfloat16 *>(p.Q) + ((int64_t)b * p.Hq + h) * D);
+                aq[ks][0] = q[(ks * 16 + 2 * t) >> 1];
+                aq[ks][2] = q[(ks * 16 + 8 + 2 * t) >> 1];
+            }
+        }
+        const float sl2 = p.inv_sqrt_d * kLog2e;
+        float Mrun = -INFINITY, lrun = 0.f;      // natural-log units, per head gi
+        float oacc[D / 8][4];
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
+
+        for (int k = 0; k < nmine; ++k) {
+            const int tau = tb + k;
+            const bool is_chunk = tau < nsel;
+            const int64_t j0 = tile_j0(tau);
+            if (!__syncthreads_and(mbar_wait(&bar[k & 1], (k >> 1) & 1, &dummy_abort) ? 1 : 0)) {
+                arrived_all = false;
+                break;
+            }
+            const uint32_t sK = smem_u32(smem + (k & 1) * 2 * TB);
+            const uint32_t sV = sK + TB;
+            float sacc[NT][4];
+#pragma unroll
+            for (int n = 0; n < NT; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+#pragma unroll
+            for (int np2 = 0; np2 < NT; np2 += 2) {
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const int hf = ks / 4;
+                    const int tok = warp * TOK_W + np2 * 8 + (lane & 7) + ((lane >> 4) << 3);
+                    const int u = (ks % 4) * 2 + ((lane >> 3) & 1);
+                    uint32_t bm[4];
+                    ldsm_x4(sK + hf * (S_TOK * 128) + swz(tok, u), bm);
+                    mma_bf16(sacc[np2], aq[ks], bm[0], bm[1]);
+                    mma_bf16(sacc[np2 + 1], aq[ks], bm[2], bm[3]);
+                }
+            }
+            float mloc = -INFINITY;
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int64_t j = j0 + warp * TOK_W + n * 8 + 2 * t + q;
+                    float x = sacc[n][q] * sl2;
+                    if (!is_chunk && (j < w0 || j > i)) x = -INFINITY;
+                    sacc[n][q] = x;
+                    mloc = fmaxf(mloc, x);
+                }
+            mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+            mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+            if (t == 0) red[warp][gi] = mloc;
+            __syncthreads();
+            const float m = fmaxf(fmaxf(red[0][gi], red[1][gi]), fmaxf(red[2][gi], red[3][gi]));
+            __syncthreads();
+            float sloc = 0.f;
+#pragma unroll
+            for (int n = 0; n < NT; ++n)
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const float e = (sacc[n][q] == -INFINITY) ? 0.f : fast_exp2(sacc[n][q] - m);
+                    sacc[n][q] = e;
+                    sloc += e;
+                }
+            sloc += __shfl_xor_sync(0xffffffffu, sloc, 1);
+            sloc += __shfl_xor_sync(0xffffffffu, sloc, 2);
+            if (t == 0) red[warp][gi] = sloc;
+            __syncthreads();
+            const float z = red[0][gi] + red[1][gi] + red[2][gi] + red[3][gi];
+            __syncthreads();
+            // this tile's weights relative to its own reference m_t:
+            // chunk tile: m_t = s^_c, weights e/z, mass 1; window: m_t = max, e, z
+            float m_t, scale_t, mass_t;
+            if (is_chunk) {
+                const int h = (gi < G) ? p.group_heads[g * G + gi] : 0;
+                m_t = (gi < G) ? p.sel[((int64_t)b * p.Hq + h) * p.K + tau] : 0.f;
+                scale_t = 1.f / z;
+                mass_t = 1.f;
+            } else {
+                m_t = m / kLog2e;
+                scale_t = 1.f;
+                mass_t = z;
+            }
+            // online merge with the running reference
+            const float Mn = fmaxf(Mrun, m_t);
+            const float fo = (Mrun == -INFINITY) ? 0.f : fast_exp2((Mrun - Mn) * kLog2e);
+            const float fn = fast_exp2((m_t - Mn) * kLog2e);
+            lrun = lrun * fo + mass_t * fn;
+            Mrun = Mn;
+#pragma unroll
+            for (int n = 0; n < D / 8; ++n) { oacc[n][0] *= fo; oacc[n][1] *= fo; }
+            const float ws = scale_t * fn;
+#pragma unroll
+            for (int kk = 0; kk < TOK_W / 16; ++kk) {
+                uint32_t ap[4];
+                ap[0] = pack_bf16(sacc[2 * kk][0] * ws, sacc[2 * kk][1] * ws);
+                ap[1] = 0u;
+                ap[2] = pack_bf16(sacc[2 * kk + 1][0] * ws, sacc[2 * kk + 1][1] * ws);
+                ap[3] = 0u;
+                if (gi >= G) ap[0] = ap[2] = 0u;
+                const int tok = warp * TOK_W + kk * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+                for (int n = 0; n < D / 8; n += 2) {
+                    const int hf = n / 8;
+                    const int u = (n % 8) + (lane >> 4);
+                    uint32_t bm[4];
+                    ldsm_x4_t(sV + hf * (S_TOK * 128) + swz(tok, u), bm);
+                    mma_bf16(oacc[n], ap, bm[0], bm[1]);
+                    mma_bf16(oacc[n + 1], ap, bm[2], bm[3]);
+                }
+            }
+            __syncthreads();                     // buffer k & 1 fully read
+            if (threadIdx.x == 0 && k + 2 < nmine) issue(k + 2);
+        }
+        if (!arrived_all) {
+            if (threadIdx.x == 0) {
+                report(p.status, HILS_ERR_DEVICE_TIMEOUT);
+                mbar_drain(&bar[0], 0);
+                mbar_drain(&bar[1], 0);
+            }
+            __syncthreads();
+            return;                              // no ticket: O stays unwritten
+        }
+        // reduce the 4 warps' O (rows gi < G; cols 8n + 2t, +1)
+        if (gi < G) {
+#pragma unroll
+            for (int n = 0; n < D / 8; ++n) {
+                ored[(warp * 8 + gi) * D + 8 * n + 2 * t] = oacc[n][0];
+                ored[(warp * 8 + gi) * D + 8 * n + 2 * t + 1] = oacc[n][1];
+            }
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < G * D; e += kAttThreads) {
+            const int hh = e / D, c = e % D;
+            float v = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) v += ored[(w * 8 + hh) * D + c];
+            p.ws_o[(((int64_t)bg * p.ntile + grp) * G + hh) * D + c] = v;
+        }
+        if (t == 0 && warp == 0 && gi < G) {
+            float *ml = p.ws_ml + (((int64_t)bg * p.ntile + grp) * G + gi) * 2;
+            ml[0] = Mrun;
+            ml[1] = lrun;
+        }
+    }
+
+    // arrival ticket; the last CTA of this (b, g) combines the groups in order
+    __threadfence();                             // this thread's partials, device-wide
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        const int prev = atomicAdd(&p.ws_cnt[bg], 1);
+        last = (prev == (int)gridDim.x - 1) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!last || !ok) return;
+    __threadfence();
+    const int ngrp = (ntot + kAttPer - 1) / kAttPer;
+    for (int e = threadIdx.x; e < G * D; e += kAttThreads) {
+        const int hh = e / D, c = e % D;
+        float M = -INFINITY;
+        for (int gg = 0; gg < ngrp; ++gg)
+            M = fmaxf(M, __ldcg(p.ws_ml + (((int64_t)bg * p.ntile + gg) * G + hh) * 2));
+        float num = 0.f, den = 0.f;
+        for (int gg = 0; gg < ngrp; ++gg) {
+            const float *ml = p.ws_ml + (((int64_t)bg * p.ntile + gg) * G + hh) * 2;
+            const float w = exp2f((__ldcg(ml) - M) * kLog2e);
+            den += w * __ldcg(ml + 1);
+            num += w * __ldcg(p.ws_o + (((int64_t)bg * p.ntile + gg) * G + hh) * D + c);
+        }
+        const int h = p.group_heads[g * G + hh];
+        reinterpret_cast<__nv_bfloat16 *>(p.O)[((int64_t)b * p.Hq + h) * D + c] =
+            __float2bfloat16_rn(num / den);
+    }
+    if (threadIdx.x == 0) p.ws_cnt[bg] = 0;      // ready for the next call
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t,
+                                  void *, const cuuint64_t *, const cuuint64_t *,
+                                  const cuuint32_t *, const cuuint32_t *,
+                                  CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion,
+                                  CUtensorMapFloatOOBfill);
+
+bool map_2d(CUtensorMap *m, const void *base, int d, int64_t rows, int box_rows) {
+    void *fp = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fp, cudaEnableDefault,
+                                &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+        return false;
+    EncodeTiledFn f = (EncodeTiledFn)fp;
+    cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return f(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims,
+             strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DecPlan {
+    int ncs, nsplit, cps, ntile;
+    size_t off_s, off_p, off_o, off_ml, off_cnt, total;
+};
+
+DecPlan dec_plan(const Problem &p) {
+    DecPlan pl;
+    int64_t w0, ncm;
+    window_bounds((int64_t)p.kv_rows - 1, p.S, p.W, &w0, &ncm);
+    pl.ncs = (int)(ncm > 0 ? ncm : 1);
+    // splits sized so that about 3 CTAs per SM stream the whole scan
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t want = (int64_t)3 * sms;
+    const int64_t per_bg = (want + (int64_t)p.B * p.Hkv - 1) / ((int64_t)p.B * p.Hkv);
+    int64_t tiles = (pl.ncs + kTileChunks - 1) / kTileChunks;
+    int64_t tps = (tiles + per_bg - 1) / (per_bg > 0 ? per_bg : 1);
+    if (tps < 4) tps = 4;
+    pl.cps = (int)(tps * kTileChunks);
+    pl.nsplit = (pl.ncs + pl.cps - 1) / pl.cps;
+    pl.ntile = p.K + (p.W + 2 * p.S - 2) / p.S + 1;
+    auto al = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t bg = (size_t)p.B * p.Hkv;
+    pl.off_s = 0;
+    pl.off_p = al(pl.off_s + sizeof(float) * bg * p.G * pl.ncs);
+    pl.off_o = al(pl.off_p + sizeof(float) * bg * pl.nsplit * p.G * 2);
+    pl.off_ml = al(pl.off_o + sizeof(float) * bg * pl.ntile * p.G * p.d);
+    pl.off_cnt = al(pl.off_ml + sizeof(float) * bg * pl.ntile * p.G * 2);
+    pl.total = al(pl.off_cnt + sizeof(int32_t) * bg);
+    return pl;
+}
+
+DecParams dec_params(const Problem &p, void *ws) {
+    DecPlan pl = dec_plan(p);
+    DecParams d;
+    char *base = (char *)ws;
+    d.Q = p.Q; d.Qs = p.Qs; d.bias = p.bias; d.cache_len = p.cache_len;
+    d.O = p.O; d.idx = p.idx; d.sel = p.sel; d.status = p.status;
+    d.ws_s = (float *)(base + pl.off_s);
+    d.ws_p = (float *)(base + pl.off_p);
+    d.ws_o = (float *)(base + pl.off_o);
+    d.ws_ml = (float *)(base + pl.off_ml);
+    d.ws_cnt = (int32_t *)(base + pl.off_cnt);
+    d.B = p.B; d.Hq = p.Hq; d.Hkv = p.Hkv; d.G = p.G; d.d = p.d; d.S = p.S;
+    d.W = p.W; d.K = p.K; d.Lmax = p.kv_rows; d.nC = p.nC;
+    d.ncs = pl.ncs; d.nsplit = pl.nsplit; d.cps = pl.cps; d.ntile = pl.ntile;
+    d.inv_sqrt_d = p.inv_sqrt_d;
+    for (int k = 0; k < kMaxHeads; ++k) d.group_heads[k] = p.group_heads[k];
+    return d;
+}
+
+}  // namespace
+
+bool dec_fast_supported(const Problem &p) {
+    if (!p.decode || p.dtype != HILS_BF16) return false;
+    if (!(p.d == 64 || p.d == 128) || !(p.S == 64 || p.S == 128)) return false;
+    if (p.G > 8 || p.nC < 1) return false;
+    int64_t w0, ncm;
+    window_bounds((int64_t)p.kv_rows - 1, p.S, p.W, &w0, &ncm);
+    if (ncm > (int64_t)kSelPer * kSelThreads) return false;
+    if ((int64_t)p.B * p.Hkv * p.kv_rows >= (1ll << 31)) return false;
+    return true;
+}
+
+size_t dec_workspace_bytes(const Problem &p) { return dec_plan(p).total; }
+
+cudaError_t launch_dec_select(Problem &p, void *ws, cudaStream_t st) {
+    DecParams d = dec_params(p, ws);
+    CUtensorMap tl;
+    if (!map_2d(&tl, p.Klm, p.d, (int64_t)p.B * p.Hkv * p.nC, kTileChunks))
+        return cudaErrorInvalidValue;
+    const size_t smem = 1024 + (size_t)kScoreStages * kTileChunks * p.d * 2;
+    dim3 grid(d.nsplit, p.Hkv, p.B);
+    cudaError_t e;
+    if (p.d == 128) {
+        e = cudaFuncSetAttribute(dec_score_kernel<128>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess)
+            dec_score_kernel<128><<<grid, kScoreWarps * 32, smem, st>>>(tl, d);
+    } else {
+        e = cudaFuncSetAttribute(dec_score_kernel<64>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess)
+            dec_score_kernel<64><<<grid, kScoreWarps * 32, smem, st>>>(tl, d);
+    }
+    if (e != cudaSuccess) return e;
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    dec_select_kernel<<<dim3(p.Hkv, p.B), kSelThreads, 0, st>>>(d);
+    count_launches(2);
+    return cudaGetLastError();
+}
+
+template <int S_TOK, int D>
+cudaError_t launch_att_t(const DecParams &d, const CUtensorMap &tk,
+                         const CUtensorMap &tv, cudaStream_t st) {
+    const size_t smem = 1024 + 4ull * S_TOK * D * 2 + 4ull * 8 * D * 4;
+    cudaError_t e = cudaFuncSetAttribute(dec_attend_kernel<S_TOK, D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int ngrp = (d.ntile + kAttPer - 1) / kAttPer;
+    dec_attend_kernel<S_TOK, D><<<dim3(ngrp, d.Hkv, d.B), kAttThreads, smem, st>>>(tk, tv, d);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dec_attend(Problem &p, void *ws, cudaStream_t st) {
+    DecParams d = dec_params(p, ws);
+    CUtensorMap tk, tv;
+    const int64_t rows = (int64_t)p.B * p.Hkv * p.kv_rows;
+    if (!map_2d(&tk, p.Kc, p.d, rows, p.S) || !map_2d(&tv, p.V, p.d, rows, p.S))
+        return cudaErrorInvalidValue;
+    cudaError_t e;
+    if (p.S == 64 && p.d == 128) e = launch_att_t<64, 128>(d, tk, tv, st);
+    else if (p.S == 64 && p.d == 64) e = launch_att_t<64, 64>(d, tk, tv, st);
+    else if (p.S == 128 && p.d == 128) e = launch_att_t<128, 128>(d, tk, tv, st);
+    else e = launch_att_t<128, 64>(d, tk, tv, st);
+    count_launches(1);
+    return e;
+}
+
+}  // namespace hils

@@ -83,10 +83,14 @@ bool attend_supported(const Problem &p) {
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n); }
 uint64_t launch_total() { return g_launches.load(); }
 
-bool fast_path_supported(const Problem &p) { return attend_supported(p); }
+bool fast_path_supported(const Problem &p) {
+    if (p.decode) return p.dtype == HILS_BF16 && encode_fn() && dec_fast_supported(p);
+    return attend_supported(p);
+}
 
 bool fast_select_supported(const Problem &p) {
-    if (p.decode || p.dtype != HILS_BF16) return false;
+    if (p.decode) return p.dtype == HILS_BF16 && encode_fn() && dec_fast_supported(p);
+    if (p.dtype != HILS_BF16) return false;
     if (!(p.d == 64 || p.d == 128)) return false;
     if (128 % p.G != 0 || p.nC < 1) return false;
     if (!encode_fn()) return false;
@@ -95,13 +99,13 @@ bool fast_select_supported(const Problem &p) {
 }
 
 size_t fast_workspace_bytes(const Problem &p) {
-    (void)p;
-    return 0;
+    return p.decode ? dec_workspace_bytes(p) : 0;
 }
 
 cudaError_t launch_fast_select(Problem &p, void *ws, size_t ws_bytes,
                                cudaStream_t st) {
-    (void)ws; (void)ws_bytes;
+    (void)ws_bytes;
+    if (p.decode) return launch_dec_select(p, ws, st);
     TcParams tp = tc_params(p);
     TcMaps maps;
     if (!make_map(&maps.lm, p.Klm, p.d, p.nC, p.Hkv, p.B, 128))
@@ -113,7 +117,8 @@ cudaError_t launch_fast_select(Problem &p, void *ws, size_t ws_bytes,
 
 cudaError_t launch_fast_attend(Problem &p, void *ws, size_t ws_bytes,
                                cudaStream_t st) {
-    (void)ws; (void)ws_bytes;
+    (void)ws_bytes;
+    if (p.decode) return launch_dec_attend(p, ws, st);
     TcParams tp = tc_params(p);
     TcMaps maps;
     if (!make_map(&maps.q, p.Q, p.d, p.n_query, p.Hq, p.B, tp.M) ||

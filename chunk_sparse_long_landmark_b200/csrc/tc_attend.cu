@@ -122,29 +122,60 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
     const int nwords = (p.nC + 31) >> 5;
     for (int w = threadIdx.x; w < nwords; w += kThreads) s_bits[w] = 0u;
     __syncthreads();
-    for (int e = threadIdx.x; e < p.M * p.K; e += kThreads) {
-        const int m = e / p.K, k = e % p.K;      // consecutive e: one row's list
-        const int i = i0 + m;
-        int c = -1;
-        if (i < p.N) {
-            int64_t w0, nc;
-            window_bounds(i, p.S, p.W, &w0, &nc);
-            c = p.idx[(((int64_t)b * p.Hkv + g) * p.N + i) * p.K + k];
-            if (c < 0 || c >= nc) c = -1;
+    // The block's idx rows are one contiguous [M][K] range, its scores G
+    // contiguous [M][K] ranges: loads are issued in batches of 8 per thread
+    // before their stores so their latencies overlap.
+    {
+        const int nidx = p.M * p.K;
+        const int32_t *gidx = p.idx + (((int64_t)b * p.Hkv + g) * p.N + i0) * p.K;
+        const int nvalid = (min(i0 + p.M, p.N) - i0) * p.K;
+        for (int e0 = 0; e0 < nidx; e0 += 8 * kThreads) {
+            int c8[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int e = e0 + q * kThreads + threadIdx.x;
+                c8[q] = (e < nvalid) ? __ldg(gidx + e) : -1;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int e = e0 + q * kThreads + threadIdx.x;
+                if (e < nidx) {
+                    const int m = e / p.K, k = e % p.K;
+                    int c = c8[q];
+                    if (c >= 0) {
+                        int64_t w0, nc;
+                        window_bounds(i0 + m, p.S, p.W, &w0, &nc);
+                        if (c >= nc) c = -1;
+                    }
+                    s_idx[k * p.M + m] = c;
+                    if (c >= 0) atomicOr(&s_bits[c >> 5], 1u << (c & 31));
+                }
+            }
         }
-        s_idx[k * p.M + m] = c;
-        if (c >= 0) atomicOr(&s_bits[c >> 5], 1u << (c & 31));
-    }
-    for (int e = threadIdx.x; e < kRows * p.K; e += kThreads) {
-        const int r = e / p.K, k = e % p.K;
-        const int hh = r / p.M, m = r % p.M;
-        const int i = i0 + m;
-        float v = -INFINITY;
-        if (i < p.N && hh < p.G) {
-            const int h = p.group_heads[g * p.G + hh];
-            v = p.sel[(((int64_t)b * p.Hq + h) * p.N + i) * p.K + k];
+        for (int e0 = 0; e0 < kRows * p.K; e0 += 8 * kThreads) {
+            float v8[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int e = e0 + q * kThreads + threadIdx.x;
+                v8[q] = -INFINITY;
+                if (e < kRows * p.K) {
+                    const int hh = e / nidx, rem = e % nidx;   // head slot, [m][k]
+                    if (rem < nvalid) {
+                        const int h = p.group_heads[g * p.G + hh];
+                        v8[q] = __ldg(p.sel + (((int64_t)b * p.Hq + h) * p.N + i0) * p.K + rem);
+                    }
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const int e = e0 + q * kThreads + threadIdx.x;
+                if (e < kRows * p.K) {
+                    const int hh = e / nidx, rem = e % nidx;
+                    const int m = rem / p.K, k = rem % p.K;
+                    s_sel[k * kRows + hh * p.M + m] = v8[q];
+                }
+            }
         }
-        s_sel[k * kRows + r] = v;
     }
     __syncthreads();
     if (warp == 0) {                       // ascending compaction of the union

@@ -29,6 +29,10 @@ struct TcMaps {
     CUtensorMap lm; // Klm [B,Hkv,nC,d]: box {64, 128, 1, 1}
 };
 
+bool dec_fast_supported(const Problem &p);
+size_t dec_workspace_bytes(const Problem &p);
+cudaError_t launch_dec_select(Problem &p, void *ws, cudaStream_t st);
+cudaError_t launch_dec_attend(Problem &p, void *ws, cudaStream_t st);
 size_t tc_score_smem_bytes(const TcParams &tp, int d);
 cudaError_t launch_tc_score(const TcParams &tp, const TcMaps &maps,
                             const void *qhat, cudaStream_t st);

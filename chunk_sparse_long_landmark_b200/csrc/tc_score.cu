@@ -161,21 +161,37 @@ tc_score_kernel(const __grid_constant__ CUtensorMap tmL, const void *qhat,
     if (warp == 1) tmem_alloc(&st.tmem_base, 256);
     if (warp == 0 && lane == 0) prefetch_tmap(&tmL);
 
-    // scoring-query tile, query-major rows, K-major 128B-swizzled halves
-    for (int e = threadIdx.x; e < kRows * (D / 8); e += kThreads) {
-        const int r = e / (D / 8), u = e % (D / 8);     // 16-byte unit u of row r
-        const int m = r / G, hh = r % G;
-        const int i = i0 + m;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (i < p.N) {
-            const int h = p.group_heads[g * G + hh];
-            v = *reinterpret_cast<const uint4 *>(
-                reinterpret_cast<const __nv_bfloat16 *>(qhat) +
-                (((int64_t)b * p.Hq + h) * p.N + i) * D + u * 8);
+    // scoring-query tile, query-major rows, K-major 128B-swizzled halves;
+    // every load is issued before the first store so they overlap
+    {
+        constexpr int kUnits = kRows * (D / 8);           // 16-byte units
+        constexpr int kPer = (kUnits + kThreads - 1) / kThreads;
+        uint4 v[kPer];
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int e = threadIdx.x + q * kThreads;
+            v[q] = make_uint4(0, 0, 0, 0);
+            if (e < kUnits) {
+                const int r = e / (D / 8), u = e % (D / 8);
+                const int i = i0 + r / G;
+                if (i < p.N) {
+                    const int h = p.group_heads[g * G + r % G];
+                    v[q] = __ldg(reinterpret_cast<const uint4 *>(
+                        reinterpret_cast<const __nv_bfloat16 *>(qhat) +
+                        (((int64_t)b * p.Hq + h) * p.N + i) * D + u * 8));
+                }
+            }
         }
-        const int half = u >> 3, uu = u & 7;
-        *reinterpret_cast<uint4 *>(smem + L::OFF_Q + half * (kRows * 128) +
-                                   r * 128 + ((uu ^ (r & 7)) << 4)) = v;
+#pragma unroll
+        for (int q = 0; q < kPer; ++q) {
+            const int e = threadIdx.x + q * kThreads;
+            if (e < kUnits) {
+                const int r = e / (D / 8), u = e % (D / 8);
+                const int half = u >> 3, uu = u & 7;
+                *reinterpret_cast<uint4 *>(smem + L::OFF_Q + half * (kRows * 128) +
+                                           r * 128 + ((uu ^ (r & 7)) << 4)) = v[q];
+            }
+        }
     }
     fence_async_smem();
     tc_fence_before();

@@ -11,8 +11,10 @@
 //   P   = softmax    per row, in registers (chunk tiles: intra-chunk softmax
 //                    scaled by exp(s^_c - M0)/z_c, zero for rows that did not
 //                    select the chunk; window tiles: causal + window mask,
-//                    running reference max)
-//   O  += P V        tcgen05.mma, 128 x d, A = P (bf16, smem), f32 in TMEM
+//                    running reference max), stored as bf16 over the S columns
+//   O  += P V        tcgen05.mma, 128 x d, A = P from TMEM, f32 in TMEM
+// Shared memory holds only Q and a 2-stage K/V ring (~105 KB) and TMEM 256
+// columns, so two CTAs share an SM and hide each other's latencies.
 // Warp roles: warp 0 TMA producer, warp 1 MMA issuer (and TMEM owner),
 // warps 2-5 softmax / epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
 // All waits are bounded (sm100::mbar_wait): a lost arrival ends the kernel
@@ -36,19 +38,17 @@ constexpr float kRescaleLog2 = 8.0f;      // lazy O rescale threshold (log2)
 
 template <int S_TOK, int D>
 struct AttnLayout {
-    static constexpr int NP = (S_TOK == 64) ? 2 : 1;           // P buffers
     static constexpr uint32_t Q_BYTES = kRows * D * 2;
     static constexpr uint32_t KV_BYTES = S_TOK * D * 2;        // one of K or V
-    static constexpr uint32_t P_BYTES = kRows * S_TOK * 2;
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
     static constexpr uint32_t OFF_V = OFF_K + kStages * KV_BYTES;
-    static constexpr uint32_t OFF_P = OFF_V + kStages * KV_BYTES;
-    static constexpr uint32_t OFF_SMALL = OFF_P + NP * P_BYTES;
+    static constexpr uint32_t OFF_SMALL = OFF_V + kStages * KV_BYTES;
     static constexpr int TMEM_O = 0;                 // columns [0, D)
-    static constexpr int TMEM_S = D;                 // 2 buffers of S_TOK
+    static constexpr int TMEM_S = D;                 // 2 buffers of S_TOK (S, then P)
     static constexpr uint32_t TMEM_COLS =
         (D + 2 * S_TOK) <= 256 ? 256u : 512u;
+    static constexpr int MIN_BLOCKS = (TMEM_COLS <= 256) ? 2 : 1;
 };
 
 struct SmallState {
@@ -56,9 +56,8 @@ struct SmallState {
     uint64_t kv_full[kStages];
     uint64_t kv_empty[kStages];
     uint64_t s_full[2];
-    uint64_t s_empty[2];
     uint64_t p_full[2];
-    uint64_t p_empty[2];
+    uint64_t p_empty[2];                             // PV of that buffer done
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort;
@@ -68,7 +67,7 @@ struct SmallState {
 };
 
 template <int S_TOK, int D>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, AttnLayout<S_TOK, D>::MIN_BLOCKS)
 tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
                  const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV,
@@ -77,11 +76,9 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     SmallState &st = *reinterpret_cast<SmallState *>(smem + L::OFF_SMALL);
-    // selected chunks of the block's queries, [K][M]; their scores for every
-    // row, [K][128]; the chunk union; its bitmap
+    // selected chunks of the block's queries, [K][M]; the chunk union; its bitmap
     int *s_idx = reinterpret_cast<int *>(smem + L::OFF_SMALL + sizeof(SmallState));
-    float *s_sel = reinterpret_cast<float *>(s_idx + p.M * p.K);
-    int *s_union = reinterpret_cast<int *>(s_sel + kRows * p.K);
+    int *s_union = s_idx + p.M * p.K;
     uint32_t *s_bits = reinterpret_cast<uint32_t *>(s_union + p.ucap);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -102,7 +99,6 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&st.s_full[s], 1);
-            mbar_init(&st.s_empty[s], 128);
             mbar_init(&st.p_full[s], 128);
             mbar_init(&st.p_empty[s], 1);
         }
@@ -149,30 +145,6 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
                     }
                     s_idx[k * p.M + m] = c;
                     if (c >= 0) atomicOr(&s_bits[c >> 5], 1u << (c & 31));
-                }
-            }
-        }
-        for (int e0 = 0; e0 < kRows * p.K; e0 += 8 * kThreads) {
-            float v8[8];
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int e = e0 + q * kThreads + threadIdx.x;
-                v8[q] = -INFINITY;
-                if (e < kRows * p.K) {
-                    const int hh = e / nidx, rem = e % nidx;   // head slot, [m][k]
-                    if (rem < nvalid) {
-                        const int h = p.group_heads[g * p.G + hh];
-                        v8[q] = __ldg(p.sel + (((int64_t)b * p.Hq + h) * p.N + i0) * p.K + rem);
-                    }
-                }
-            }
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int e = e0 + q * kThreads + threadIdx.x;
-                if (e < kRows * p.K) {
-                    const int hh = e / nidx, rem = e % nidx;
-                    const int m = rem / p.K, k = rem % p.K;
-                    s_sel[k * kRows + hh * p.M + m] = v8[q];
                 }
             }
         }
@@ -262,22 +234,20 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
             const uint32_t sQ = smem_u32(smem + L::OFF_Q);
             const uint32_t sK = smem_u32(smem + L::OFF_K);
             const uint32_t sV = smem_u32(smem + L::OFF_V);
-            const uint32_t sP = smem_u32(smem + L::OFF_P);
             bool ok = mbar_wait(&st.q_full, 0, abort);
             tc_fence_after();
             auto do_pv = [&](int u) -> bool {
-                const int pb = u % L::NP;
-                if (!mbar_wait(&st.p_full[pb], (u / L::NP) & 1, abort)) return false;
+                const int pb = u & 1;
+                if (!mbar_wait(&st.p_full[pb], (u >> 1) & 1, abort)) return false;
                 tc_fence_after();
                 const int s = u % kStages;
 #pragma unroll
                 for (int k = 0; k < S_TOK / 16; ++k) {
-                    const uint64_t ad = desc_sw128(
-                        sP + pb * L::P_BYTES + (k / 4) * (kRows * 128) + (k % 4) * 32,
-                        16, 1024);
+                    // A = P of this tile, bf16 in the S buffer: 8 columns per 16 tokens
+                    const uint32_t at = tmem + L::TMEM_S + pb * S_TOK + k * 8;
                     const uint64_t bd = desc_sw128(
                         sV + s * L::KV_BYTES + k * 16 * 128, S_TOK * 128, 1024);
-                    mma_ss(tmem + L::TMEM_O, ad, bd, id_o, (u > 0 || k > 0) ? 1u : 0u);
+                    mma_ts(tmem + L::TMEM_O, at, bd, id_o, (u > 0 || k > 0) ? 1u : 0u);
                 }
                 mma_commit(&st.kv_empty[s]);
                 mma_commit(&st.p_empty[pb]);
@@ -287,7 +257,8 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
                 const int s = t % kStages;
                 const int sb = t & 1;
                 if (!mbar_wait(&st.kv_full[s], (t / kStages) & 1, abort)) { ok = false; break; }
-                if (t >= 2 && !mbar_wait(&st.s_empty[sb], ((t >> 1) - 1) & 1, abort)) { ok = false; break; }
+                // S buffer sb is free once PV(t-2), which read its P, is done
+                if (t >= 2 && !mbar_wait(&st.p_empty[sb], ((t - 2) >> 1) & 1, abort)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
@@ -317,19 +288,20 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
         int64_t w0 = 0, nc = 0;
         if (valid) window_bounds(i, p.S, p.W, &w0, &nc);
         const int *myidx = s_idx + m;                    // stride M
-        const float *mysel = s_sel + r;                  // stride 128
         const int M_ = p.M;
+        const float *mysel = p.sel + (((int64_t)b * p.Hq + h) * p.N + i) * p.K;
         float M0 = -INFINITY;                            // natural-log units
         if (valid)
             for (int k = 0; k < p.K; ++k)
-                if (myidx[k * M_] >= 0) M0 = fmaxf(M0, mysel[k * kRows]);
+                if (myidx[k * M_] >= 0) M0 = fmaxf(M0, __ldg(mysel + k));
         const float M0l2 = M0 * kLog2e;
         float mref = M0l2;                               // log2 units
         float l = 0.f;
         int kp = 0;
+        // s^ of the next selected chunk, loaded ahead of its tile
+        float sh_next = (valid && p.K > 0) ? __ldg(mysel) : 0.f;
         const float sl2 = p.inv_sqrt_d * kLog2e;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-        uint8_t *sP = smem + L::OFF_P;
         bool ok = true;
 
         for (int t = 0; t < T; ++t) {
@@ -347,17 +319,20 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
                 for (int j = 0; j < 32; ++j) x[c0 + j] = __uint_as_float(rr[j]) * sl2;
             }
-            tc_fence_before();
-            mbar_arrive(&st.s_empty[sb]);
 
             if (t < U) {
                 const int c = s_union[t];
                 int ck = kp < p.K ? myidx[kp * M_] : 0x7fffffff;
-                while (kp < p.K && ck < c) { ++kp; ck = kp < p.K ? myidx[kp * M_] : 0x7fffffff; }
+                while (kp < p.K && ck < c) {
+                    ++kp;
+                    ck = kp < p.K ? myidx[kp * M_] : 0x7fffffff;
+                    sh_next = (valid && kp < p.K) ? __ldg(mysel + kp) : 0.f;
+                }
                 const bool sel = valid && kp < p.K && ck == c;
                 if (sel) {
-                    const float sh = mysel[kp * kRows] * kLog2e;
+                    const float sh = sh_next * kLog2e;
                     ++kp;
+                    sh_next = (kp < p.K) ? __ldg(mysel + kp) : 0.f;
                     float mc = x[0];
 #pragma unroll
                     for (int j = 1; j < S_TOK; ++j) mc = fmaxf(mc, x[j]);
@@ -392,7 +367,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
                                     : (mref == -INFINITY) ? 0.f : fast_exp2(mref - mx);
                     if (t >= 1) {
                         const int u = t - 1;
-                        if (!__all_sync(0xffffffffu, mbar_wait(&st.p_empty[u % L::NP], (u / L::NP) & 1, abort))) { ok = false; break; }
+                        if (!__all_sync(0xffffffffu, mbar_wait(&st.p_empty[u & 1], (u >> 1) & 1, abort))) { ok = false; break; }
                         tc_fence_after();
 #pragma unroll
                         for (int c0 = 0; c0 < D; c0 += 32) {
@@ -417,36 +392,23 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
                 l += es;
             }
 
-            // P -> smem (bf16, K-major, 128B swizzle), then hand to the MMA
-            const int pb = t % L::NP;
-            if (t >= L::NP) {
-                const int u = t - L::NP;
-                if (!__all_sync(0xffffffffu, mbar_wait(&st.p_empty[pb], (u / L::NP) & 1, abort))) { ok = false; break; }
-            }
-            uint8_t *prow = sP + pb * L::P_BYTES + r * 128;
+            // P -> TMEM over this tile's S columns (bf16 pairs), then the MMA
 #pragma unroll
-            for (int half = 0; half < S_TOK / 64; ++half) {
+            for (int c0 = 0; c0 < S_TOK; c0 += 64) {
+                uint32_t pk[32];
 #pragma unroll
-                for (int uu = 0; uu < 8; ++uu) {
-                    const int j = half * 64 + uu * 8;
-                    uint4 v;
-                    v.x = pack_bf16(x[j + 0], x[j + 1]);
-                    v.y = pack_bf16(x[j + 2], x[j + 3]);
-                    v.z = pack_bf16(x[j + 4], x[j + 5]);
-                    v.w = pack_bf16(x[j + 6], x[j + 7]);
-                    *reinterpret_cast<uint4 *>(prow + half * (kRows * 128) +
-                                               ((uu ^ (r & 7)) << 4)) = v;
-                }
+                for (int j = 0; j < 32; ++j) pk[j] = pack_bf16(x[c0 + 2 * j], x[c0 + 2 * j + 1]);
+                tmem_st32(trow + L::TMEM_S + sb * S_TOK + c0 / 2, pk);
             }
-            fence_async_smem();
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&st.p_full[pb]);
+            mbar_arrive(&st.p_full[sb]);
         }
 
         // final: O / l once the last PV is done
         if (ok && T > 0) {
             const int u = T - 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(&st.p_empty[u % L::NP], (u / L::NP) & 1, abort));
+            ok = __all_sync(0xffffffffu, mbar_wait(&st.p_empty[u & 1], (u >> 1) & 1, abort));
         }
         if (ok) {
             tc_fence_after();
@@ -493,6 +455,9 @@ cudaError_t launch_attend_t(const TcParams &tp, const TcMaps &maps,
     cudaError_t e = cudaFuncSetAttribute(
         kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     const int nqb = (tp.N + tp.M - 1) / tp.M;
     const int64_t grid = (int64_t)tp.B * tp.Hkv * nqb;
     if (grid <= 0) return cudaSuccess;
@@ -504,11 +469,8 @@ cudaError_t launch_attend_t(const TcParams &tp, const TcMaps &maps,
 }  // namespace
 
 size_t tc_attend_smem_bytes(const TcParams &tp, int s_tok, int d) {
-    const int np = (s_tok == 64) ? 2 : 1;
-    size_t big = (size_t)kRows * d * 2 + 2ull * kStages * s_tok * d * 2 +
-                 (size_t)np * kRows * s_tok * 2;
+    size_t big = (size_t)kRows * d * 2 + 2ull * kStages * s_tok * d * 2;
     size_t small = sizeof(SmallState) + sizeof(int) * ((size_t)tp.M * tp.K + tp.ucap) +
-                   sizeof(float) * (size_t)kRows * tp.K +
                    sizeof(uint32_t) * (((size_t)tp.nC + 31) / 32);
     return 1024 + big + ((small + 15) / 16) * 16;
 }

@@ -285,6 +285,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the decode step (prints its object)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -322,6 +324,15 @@ def main():
         return float(t.item())
 
     peaks = measured_peaks()
+    if args.decode_only:
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        d = bench_decode(args, dev, torch.cuda.current_stream(dev), flush,
+                         world, max_over_ranks, barrier, rank, peaks)
+        if rank == 0:
+            print(json.dumps({"decode": d}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return
     inp = synth.make_prefill(sh, seed=synth.seed_for(cfg_id) + 17 * rank,
                              device=dev)
     work = prefill_work(sh)

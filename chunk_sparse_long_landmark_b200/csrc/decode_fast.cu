@@ -56,6 +56,7 @@ struct DecParams {
     int nsplit;         // landmark splits per (b, g)
     int cps;            // chunks per split (multiple of kTileChunks)
     int ntile;          // attention tiles per (b, g): K + window tiles
+    int att_per;        // attention tiles per CTA
     float inv_sqrt_d;
     int16_t group_heads[kMaxHeads];
 };
@@ -166,8 +167,20 @@ dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
     const float *bias = p.bias + (int64_t)bg * p.nC;
     float *outs = p.ws_s + (int64_t)bg * G * p.ncs;
     volatile int dummy_abort = 0;
+    // bias of the lane's 2 chunks of the next tile, loaded a tile ahead
+    auto load_bias = [&](int tt, float *bv) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int c = c_begin + tt * kTileChunks + warp * 16 + gi + q * 8;
+            bv[q] = (tt < ntiles && c < c_end) ? __ldg(bias + c) : 0.f;
+        }
+    };
+    float bnext[2];
+    load_bias(0, bnext);
     for (int tt = 0; tt < ntiles; ++tt) {
         const int s = tt % kScoreStages;
+        const float bcur[2] = {bnext[0], bnext[1]};
+        load_bias(tt + 1, bnext);
         mbar_wait(&full[s], (tt / kScoreStages) & 1, &dummy_abort);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
         const uint32_t base = smem_u32(smem + s * STAGE);
@@ -193,7 +206,7 @@ dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
             const int hh = 2 * t + (q & 1);
             const int c = c_begin + tt * kTileChunks + warp * 16 + gi + (q >> 1) * 8;
             if (hh < G && c < c_end) {
-                const float shat = fmaf(acc[q], p.inv_sqrt_d, bias[c]);
+                const float shat = fmaf(acc[q], p.inv_sqrt_d, bcur[q >> 1]);
                 outs[(int64_t)hh * p.ncs + c] = shat;
                 const float x = shat * kLog2e;
                 const int k = q & 1;
@@ -422,7 +435,7 @@ dec_select_kernel(const DecParams p) {
 // CTA streams its tiles through a double-buffered TMA pipeline and merges
 // them online per head: running reference max M, O accumulated in the MMA
 // registers (rescaled when M rises), l in registers.
-constexpr int kAttPer = 6;                       // tiles per CTA
+constexpr int kAttPerMin = 4;                    // tiles per CTA, at least
 
 template <int S_TOK, int D>
 __global__ void __launch_bounds__(kAttThreads)
@@ -451,8 +464,8 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
         for (int k = 0; k < p.K; ++k) nsel += (p.idx[(int64_t)bg * p.K + k] >= 0) ? 1 : 0;
     const int nwin = ok ? (int)((i - w0 + 1 + S_TOK - 1) / S_TOK) : 0;
     const int ntot = nsel + nwin;
-    const int tb = grp * kAttPer;
-    const int te = min(tb + kAttPer, ntot);
+    const int tb = grp * p.att_per;
+    const int te = min(tb + p.att_per, ntot);
     const int nmine = te > tb ? te - tb : 0;
     auto tile_j0 = [&](int tau) -> int64_t {
         return tau < nsel ? (int64_t)p.idx[(int64_t)bg * p.K + tau] * p.S
@@ -645,7 +658,7 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     __syncthreads();
     if (!last || !ok) return;
     __threadfence();
-    const int ngrp = (ntot + kAttPer - 1) / kAttPer;
+    const int ngrp = (ntot + p.att_per - 1) / p.att_per;
     for (int e = threadIdx.x; e < G * D; e += kAttThreads) {
         const int hh = e / D, c = e % D;
         float M = -INFINITY;
@@ -690,7 +703,7 @@ bool map_2d(CUtensorMap *m, const void *base, int d, int64_t rows, int box_rows)
 }
 
 struct DecPlan {
-    int ncs, nsplit, cps, ntile;
+    int ncs, nsplit, cps, ntile, att_per;
     size_t off_s, off_p, off_o, off_ml, off_cnt, total;
 };
 
@@ -703,14 +716,25 @@ DecPlan dec_plan(const Problem &p) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // one wave: at most 3 resident CTAs per SM (65 KB of stages each)
     const int64_t want = (int64_t)3 * sms;
-    const int64_t per_bg = (want + (int64_t)p.B * p.Hkv - 1) / ((int64_t)p.B * p.Hkv);
+    int64_t per_bg = want / ((int64_t)p.B * p.Hkv);
+    if (per_bg < 1) per_bg = 1;
     int64_t tiles = (pl.ncs + kTileChunks - 1) / kTileChunks;
     int64_t tps = (tiles + per_bg - 1) / (per_bg > 0 ? per_bg : 1);
     if (tps < 4) tps = 4;
     pl.cps = (int)(tps * kTileChunks);
     pl.nsplit = (pl.ncs + pl.cps - 1) / pl.cps;
     pl.ntile = p.K + (p.W + 2 * p.S - 2) / p.S + 1;
+    // attention: one wave of CTAs (2 resident per SM at S = 64, 1 at S = 128)
+    {
+        const int64_t slots = (int64_t)sms * (p.S == 64 ? 2 : 1);
+        int64_t groups = slots / ((int64_t)p.B * p.Hkv);
+        if (groups < 1) groups = 1;
+        int per = (int)((pl.ntile + groups - 1) / groups);
+        if (per < kAttPerMin) per = kAttPerMin;
+        pl.att_per = per;
+    }
     auto al = [](size_t x) { return (x + 255) / 256 * 256; };
     const size_t bg = (size_t)p.B * p.Hkv;
     pl.off_s = 0;
@@ -736,6 +760,7 @@ DecParams dec_params(const Problem &p, void *ws) {
     d.B = p.B; d.Hq = p.Hq; d.Hkv = p.Hkv; d.G = p.G; d.d = p.d; d.S = p.S;
     d.W = p.W; d.K = p.K; d.Lmax = p.kv_rows; d.nC = p.nC;
     d.ncs = pl.ncs; d.nsplit = pl.nsplit; d.cps = pl.cps; d.ntile = pl.ntile;
+    d.att_per = pl.att_per;
     d.inv_sqrt_d = p.inv_sqrt_d;
     for (int k = 0; k < kMaxHeads; ++k) d.group_heads[k] = p.group_heads[k];
     return d;
@@ -791,7 +816,7 @@ cudaError_t launch_att_t(const DecParams &d, const CUtensorMap &tk,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const int ngrp = (d.ntile + kAttPer - 1) / kAttPer;
+    const int ngrp = (d.ntile + d.att_per - 1) / d.att_per;
     dec_attend_kernel<S_TOK, D><<<dim3(ngrp, d.Hkv, d.B), kAttThreads, smem, st>>>(tk, tv, d);
     return cudaGetLastError();
 }

@@ -194,6 +194,35 @@ def measured_peaks():
                 src="fallback")
 
 
+def profiled_traffic(kernels, workload):
+    """DRAM bytes per launch that one ncu capture recorded for `kernels`.
+
+    Read from profiles/traffic.json (written from `ncu --set full` captures,
+    one launch per kernel, dram__bytes_read.sum + dram__bytes_write.sum).
+    Returns None when a kernel was not captured on this workload, or when
+    its source file has changed since the capture (sha256 prefix differs).
+    """
+    import hashlib
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        tab = json.load(open(p))
+    except (OSError, ValueError):
+        return None
+    total = 0
+    for k in kernels:
+        ent = tab.get(k)
+        if not ent or ent.get("workload") != workload:
+            return None
+        try:
+            src = open(os.path.join(ROOT, ent["file"]), "rb").read()
+        except OSError:
+            return None
+        if hashlib.sha256(src).hexdigest()[:16] != ent["source_sha256"]:
+            return None
+        total += int(ent["bytes_per_launch"])
+    return total
+
+
 # -------------------------------------------------------------- oracle arm
 def oracle_sample(inp, budget_s, positions_per_batch=8, seed=0,
                   max_batches=None):
@@ -393,7 +422,10 @@ def main():
     roof = {"bound": "tensor", "kernel": dom, "achieved": achieved,
             "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "peak_source": peaks["src"],
-            "algorithmic_flops_per_launch": dom_flops, "traffic": None}
+            "algorithmic_flops_per_launch": dom_flops,
+            "traffic": profiled_traffic(
+                ["tc_attend" if dom == "attend" else "tc_score"],
+                args.workload)}
 
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s",
@@ -547,7 +579,11 @@ def bench_decode(args, dev, stream, flush, world, max_over_ranks, barrier,
         "roofline": {"bound": "hbm", "kernel": "whole decode step (graph)",
                      "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": ach / peaks["hbm"], "peak_source": peaks["src"],
-                     "algorithmic_bytes_per_step": nbytes, "traffic": None},
+                     "algorithmic_bytes_per_step": nbytes,
+                     "traffic": profiled_traffic(["dec_score", "dec_attend"],
+                                                 name),
+                     "traffic_covers": "dec_score + dec_attend launches "
+                                       "(dec_select not captured)"},
         "config": {"B": sh.B, "Hq": sh.Hq, "Hkv": sh.Hkv, "d": sh.d,
                    "L": sh.N, "S": sh.S, "W": sh.W, "K": sh.K,
                    "l2": "flushed before every timed step"},

@@ -572,23 +572,24 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
             const float z = red[0][gi] + red[1][gi] + red[2][gi] + red[3][gi];
             __syncthreads();
             // this tile's weights relative to its own reference m_t:
-            // chunk tile: m_t = s^_c, weights e/z, mass 1; window: m_t = max, e, z
-            float m_t, scale_t, mass_t;
+            // chunk tile: m_t = s^_c, weights e/z; window: m_t = max, weights e
+            float m_t, scale_t;
             if (is_chunk) {
                 const int h = (gi < G) ? p.group_heads[g * G + gi] : 0;
                 m_t = (gi < G) ? p.sel[((int64_t)b * p.Hq + h) * p.K + tau] : 0.f;
                 scale_t = 1.f / z;
-                mass_t = 1.f;
             } else {
                 m_t = m / kLog2e;
                 scale_t = 1.f;
-                mass_t = z;
             }
             // online merge with the running reference
             const float Mn = fmaxf(Mrun, m_t);
             const float fo = (Mrun == -INFINITY) ? 0.f : fast_exp2((Mrun - Mn) * kLog2e);
             const float fn = fast_exp2((m_t - Mn) * kLog2e);
-            lrun = lrun * fo + mass_t * fn;
+            // lrun: this lane's share of the normaliser, summed from the
+            // rounded weights the MMA consumes (reduced over lanes / warps
+            // at the end), so the weights applied to V add up to one
+            lrun *= fo;
             Mrun = Mn;
 #pragma unroll
             for (int n = 0; n < D / 8; ++n) { oacc[n][0] *= fo; oacc[n][1] *= fo; }
@@ -601,6 +602,8 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                 ap[2] = pack_bf16(sacc[2 * kk + 1][0] * ws, sacc[2 * kk + 1][1] * ws);
                 ap[3] = 0u;
                 if (gi >= G) ap[0] = ap[2] = 0u;
+                lrun += (__uint_as_float(ap[0] << 16) + __uint_as_float(ap[0] & 0xffff0000u)) +
+                        (__uint_as_float(ap[2] << 16) + __uint_as_float(ap[2] & 0xffff0000u));
                 const int tok = warp * TOK_W + kk * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
 #pragma unroll
                 for (int n = 0; n < D / 8; n += 2) {
@@ -624,7 +627,10 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
             __syncthreads();
             return;                              // no ticket: O stays unwritten
         }
-        // reduce the 4 warps' O (rows gi < G; cols 8n + 2t, +1)
+        // reduce the 4 warps' O (rows gi < G; cols 8n + 2t, +1) and l
+        lrun += __shfl_xor_sync(0xffffffffu, lrun, 1);
+        lrun += __shfl_xor_sync(0xffffffffu, lrun, 2);
+        if (t == 0) red[warp][gi] = lrun;
         if (gi < G) {
 #pragma unroll
             for (int n = 0; n < D / 8; ++n) {
@@ -643,7 +649,7 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
         if (t == 0 && warp == 0 && gi < G) {
             float *ml = p.ws_ml + (((int64_t)bg * p.ntile + grp) * G + gi) * 2;
             ml[0] = Mrun;
-            ml[1] = lrun;
+            ml[1] = red[0][gi] + red[1][gi] + red[2][gi] + red[3][gi];
         }
     }
 

@@ -107,10 +107,22 @@ cudaError_t launch_fast_select(Problem &p, void *ws, size_t ws_bytes,
     (void)ws_bytes;
     if (p.decode) return launch_dec_select(p, ws, st);
     TcParams tp = tc_params(p);
-    TcMaps maps;
-    if (!make_map(&maps.lm, p.Klm, p.d, p.nC, p.Hkv, p.B, 128))
-        return cudaErrorInvalidValue;
-    cudaError_t e = launch_tc_score(tp, maps, p.Qs ? p.Qs : p.Q, st);
+    const void *qhat = p.Qs ? p.Qs : p.Q;
+    cudaError_t e;
+    if (tc_select_supported(tp)) {
+        // one thread per query, all heads of the group in its TMEM lane
+        CUtensorMap lm32, q128;
+        if (!make_map(&lm32, p.Klm, p.d, p.nC, p.Hkv, p.B, 32) ||
+            !make_map(&q128, qhat, p.d, p.n_query, p.Hq, p.B, 128))
+            return cudaErrorInvalidValue;
+        e = launch_tc_select(tp, lm32, q128, st);
+    } else {
+        // wider groups (G > 4) or K > 32: per-row heaps
+        TcMaps maps;
+        if (!make_map(&maps.lm, p.Klm, p.d, p.nC, p.Hkv, p.B, 128))
+            return cudaErrorInvalidValue;
+        e = launch_tc_score(tp, maps, qhat, st);
+    }
     count_launches(1);
     return e;
 }

@@ -339,9 +339,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
                     float z = 0.f;
 #pragma unroll
                     for (int j = 0; j < S_TOK; ++j) { x[j] = fast_exp2(x[j] - mc); z += x[j]; }
-                    const float wc = fast_exp2(sh - M0l2);
-                    l += wc;
-                    const float f = wc / z;
+                    const float f = fast_exp2(sh - M0l2) / z;
 #pragma unroll
                     for (int j = 0; j < S_TOK; ++j) x[j] *= f;
                 } else {
@@ -383,23 +381,28 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
                     }
                     if (mine) { l *= fac; mref = mx; }
                 }
-                float es = 0.f;
 #pragma unroll
-                for (int j = 0; j < S_TOK; ++j) {
+                for (int j = 0; j < S_TOK; ++j)
                     x[j] = (x[j] == -INFINITY) ? 0.f : fast_exp2(x[j] - mref);
-                    es += x[j];
-                }
-                l += es;
             }
 
-            // P -> TMEM over this tile's S columns (bf16 pairs), then the MMA
+            // P -> TMEM over this tile's S columns (bf16 pairs), then the MMA.
+            // The normaliser l sums the rounded weights the MMA consumes, so
+            // the weights applied to V add up to one: in a peaked row the
+            // rounding of P then moves O by ~2^-9 w(1-w)|v| instead of
+            // ~2^-9 w|v|.
+            float ps = 0.f;
 #pragma unroll
             for (int c0 = 0; c0 < S_TOK; c0 += 64) {
                 uint32_t pk[32];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) pk[j] = pack_bf16(x[c0 + 2 * j], x[c0 + 2 * j + 1]);
+                for (int j = 0; j < 32; ++j) {
+                    pk[j] = pack_bf16(x[c0 + 2 * j], x[c0 + 2 * j + 1]);
+                    ps += __uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u);
+                }
                 tmem_st32(trow + L::TMEM_S + sb * S_TOK + c0 / 2, pk);
             }
+            l += ps;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&st.p_full[sb]);

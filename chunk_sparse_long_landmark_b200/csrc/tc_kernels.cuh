@@ -33,6 +33,9 @@ bool dec_fast_supported(const Problem &p);
 size_t dec_workspace_bytes(const Problem &p);
 cudaError_t launch_dec_select(Problem &p, void *ws, cudaStream_t st);
 cudaError_t launch_dec_attend(Problem &p, void *ws, cudaStream_t st);
+bool tc_select_supported(const TcParams &tp);
+cudaError_t launch_tc_select(const TcParams &tp, const CUtensorMap &lm32,
+                             const CUtensorMap &q128, cudaStream_t st);
 size_t tc_score_smem_bytes(const TcParams &tp, int d);
 cudaError_t launch_tc_score(const TcParams &tp, const TcMaps &maps,
                             const void *qhat, cudaStream_t st);

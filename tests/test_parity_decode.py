@@ -36,6 +36,17 @@ def test_decode_small(name, cuda_device):
     parity.check_decode(inp, O, idx)
 
 
+def test_decode_peaked(cuda_device):
+    """Query scaled by 4 (exact in bf16): near one-hot attention, where the
+    rounding of the weights to bf16 matters most for the output error."""
+    sh = synth.Shape("bf16", 2, 32, 8, 128, 16384, 64, 512, 32)
+    inp = synth.make_decode(sh, seed=203, device=cuda_device,
+                            cache_len=[16384, 7001])
+    inp = dict(inp, Q=inp["Q"] * 4)
+    O, idx = run_decode(inp)
+    parity.check_decode(inp, O, idx)
+
+
 def test_decode_config4_full(cuda_device):
     """Batch of 8 sequences with 512K-token caches, every sequence checked."""
     sh = synth.DECODE_CONFIGS[4]

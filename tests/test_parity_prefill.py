@@ -45,6 +45,8 @@ SMALL = {
     "bf16_no_candidates": (synth.Shape("bf16", 1, 4, 1, 128, 200, 64, 512, 4), None),
     "bf16_single_token": (synth.Shape("bf16", 1, 4, 1, 128, 1, 64, 16, 2), None),
     "bf16_ragged_tail": (synth.Shape("bf16", 1, 8, 2, 128, 2111, 64, 190, 7), [0, 1, 0, 1, 0, 1, 0, 1]),
+    "bf16_g2_d64_k24": (synth.Shape("bf16", 1, 4, 2, 64, 5000, 64, 256, 24), None),
+    "bf16_g4_k32_temperature": (synth.Shape("bf16", 1, 8, 2, 128, 6000, 64, 300, 32, "temperature"), None),
 }
 
 
@@ -116,3 +118,35 @@ def test_full_size_config_sampled(cfg, cuda_device):
     assert bool((cnt == torch.clamp(nc, max=sh.K).view(1, 1, -1)).all())
     d = idx[..., 1:] - idx[..., :-1]
     assert bool(((d > 0) | ~valid[..., 1:]).all())
+
+
+@pytest.mark.parametrize("K", [5, 16, 32])
+def test_exact_score_ties_take_lower_chunks(K, cuda_device):
+    """Identical landmark keys; b' = 0 on even chunks and -1 on odd ones.
+    Every even chunk has the same group score (exactly, in any precision),
+    above every odd one, so the tie rule alone decides: idx must be the
+    lowest even chunks of C_i, then the lowest odd ones, bit for bit. Long
+    runs of equal scores also overflow any fixed-size candidate list, which
+    this checks as well."""
+    sh = synth.Shape("bf16", 1, 8, 2, 128, 9000, 64, 256, K)
+    inp = synth.make_prefill(sh, seed=77, device=cuda_device)
+    nC = sh.N // sh.S
+    klm = inp["Klm"][:, :, :1, :].expand(-1, -1, nC, -1).contiguous()
+    bias = torch.zeros(sh.B, sh.Hkv, nC, dtype=torch.float32,
+                       device=cuda_device)
+    bias[:, :, 1::2] = -1.0
+    inp = dict(inp, Klm=klm, bias=bias)
+    O, idx, _ = run_prefill(inp)
+    i = np.arange(sh.N)
+    nc = np.maximum((i - sh.W + 1) // sh.S, 0)
+    want = np.full((sh.N, K), -1, dtype=np.int32)
+    for r in range(sh.N):
+        c = np.arange(nc[r])
+        order = np.concatenate([c[0::2], c[1::2]])[:K]
+        want[r, :len(order)] = np.sort(order)
+    got = idx.cpu().numpy()
+    for b in range(sh.B):
+        for g in range(sh.Hkv):
+            np.testing.assert_array_equal(got[b, g], want)
+    parity.check_prefill(inp, O, idx,
+                         positions=parity.sample_positions(sh, n_random=16))

@@ -56,7 +56,7 @@ bool make_map(CUtensorMap *m, const void *base, int d, int64_t rows, int d2,
 
 TcParams tc_params(const Problem &p) {
     TcParams t;
-    t.Klm = p.Klm; t.bias = p.bias; t.O = p.O; t.idx = p.idx; t.sel = p.sel;
+    t.Q = p.Q; t.Klm = p.Klm; t.bias = p.bias; t.O = p.O; t.idx = p.idx; t.sel = p.sel;
     t.status = p.status;
     t.B = p.B; t.Hq = p.Hq; t.Hkv = p.Hkv; t.G = p.G; t.N = p.n_query;
     t.d = p.d; t.S = p.S; t.W = p.W; t.K = p.K; t.nC = p.nC;
@@ -133,8 +133,7 @@ cudaError_t launch_fast_attend(Problem &p, void *ws, size_t ws_bytes,
     if (p.decode) return launch_dec_attend(p, ws, st);
     TcParams tp = tc_params(p);
     TcMaps maps;
-    if (!make_map(&maps.q, p.Q, p.d, p.n_query, p.Hq, p.B, tp.M) ||
-        !make_map(&maps.k, p.Kc, p.d, p.kv_rows, p.Hkv, p.B, p.S) ||
+    if (!make_map(&maps.k, p.Kc, p.d, p.kv_rows, p.Hkv, p.B, p.S) ||
         !make_map(&maps.v, p.V, p.d, p.kv_rows, p.Hkv, p.B, p.S))
         return cudaErrorInvalidValue;
     cudaError_t e = launch_tc_attend(tp, maps, st);

@@ -4,19 +4,22 @@
 // RQ2 display) and Sec. 4.2 (M adjacent queries x G heads share one tile).
 //
 // One CTA owns 128 rows = the G query heads of one kv group x M = 128/G
-// adjacent queries (row r = head_slot * M + query_slot). It loads the union
+// adjacent queries (row r = query_slot * G + head_slot). It loads the union
 // of the M queries' selected chunks once and then every tile of the aligned
 // window the block touches, each tile S tokens of K and V brought in by TMA:
 //   S   = Q K^T      tcgen05.mma, 128 x S_TOK, f32 accumulator in TMEM
 //   P   = softmax    per row, in registers (chunk tiles: intra-chunk softmax
 //                    scaled by exp(s^_c - M0)/z_c, zero for rows that did not
-//                    select the chunk; window tiles: causal + window mask,
-//                    running reference max), stored as bf16 over the S columns
+//                    select the chunk -- a warp whose queries all skipped it
+//                    stores zeros without reading S; window tiles: causal +
+//                    window mask, running reference max), stored as bf16 over
+//                    the S columns
 //   O  += P V        tcgen05.mma, 128 x d, A = P from TMEM, f32 in TMEM
 // Shared memory holds only Q and a 2-stage K/V ring (~105 KB) and TMEM 256
 // columns, so two CTAs share an SM and hide each other's latencies.
-// Warp roles: warp 0 TMA producer, warp 1 MMA issuer (and TMEM owner),
-// warps 2-5 softmax / epilogue (warp w reads TMEM lanes 32*(w%4)..+31).
+// Warp roles: warp 0 TMA producer (K, V), warp 1 MMA issuer (and TMEM
+// owner), warps 2-5 Q loader, softmax and epilogue (warp w reads TMEM lanes
+// 32*(w%4)..+31). Elementwise softmax arithmetic uses packed f32x2 ops.
 // All waits are bounded (sm100::mbar_wait): a lost arrival ends the kernel
 // with HILS_ERR_DEVICE_TIMEOUT in the status word.
 #include <math.h>
@@ -68,8 +71,7 @@ struct SmallState {
 
 template <int S_TOK, int D>
 __global__ void __launch_bounds__(kThreads, AttnLayout<S_TOK, D>::MIN_BLOCKS)
-tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
-                 const __grid_constant__ CUtensorMap tmK,
+tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV,
                  const TcParams p) {
     using L = AttnLayout<S_TOK, D>;
@@ -92,7 +94,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
 
     // ---------------------------------------------------------- prologue
     if (threadIdx.x == 0) {
-        mbar_init(&st.q_full, 1);
+        mbar_init(&st.q_full, 128);             // the softmax threads load Q
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&st.kv_full[s], 1);
             mbar_init(&st.kv_empty[s], 1);
@@ -110,7 +112,6 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
     }
     if (warp == 1) tmem_alloc(&st.tmem_base, L::TMEM_COLS);
     if (warp == 0 && lane == 0) {
-        prefetch_tmap(&tmQ);
         prefetch_tmap(&tmK);
         prefetch_tmap(&tmV);
     }
@@ -191,14 +192,6 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
     } else if (warp == 0) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
-            mbar_expect_tx(&st.q_full, L::Q_BYTES);
-            for (int hh = 0; hh < p.G; ++hh) {
-                const int h = p.group_heads[g * p.G + hh];
-                for (int dh = 0; dh < D / 64; ++dh)
-                    tma_load_4d(smem + L::OFF_Q + dh * (kRows * 128) +
-                                    hh * p.M * 128,
-                                &tmQ, &st.q_full, dh * 64, i0, h, b);
-            }
             int issued = 0;
             for (int t = 0; t < T; ++t) {
                 const int s = t % kStages;
@@ -220,7 +213,6 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
             }
             // on abort: let the copies already issued land before exiting
             if (*abort) {
-                mbar_drain(&st.q_full, 0);
                 for (int t = (issued > kStages ? issued - kStages : 0);
                      t < issued; ++t)
                     mbar_drain(&st.kv_full[t % kStages], (t / kStages) & 1);
@@ -279,14 +271,52 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
     } else {
         // -------------------------------------------- softmax / epilogue
+        // Query-major rows: row r = query_slot * G + head_slot, so a warp
+        // holds 32 / G whole queries and can skip, as a unit, every union
+        // chunk none of them selected.
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
-        const int hh = r / p.M, m = r % p.M;
+        const int m = r / p.G, hh = r % p.G;
         const int i = i0 + m;
-        const bool valid = (hh < p.G) && (i < p.N);
-        const int h = valid ? p.group_heads[g * p.G + hh] : 0;
+        const bool valid = i < p.N;
+        const int h = p.group_heads[g * p.G + hh];
         int64_t w0 = 0, nc = 0;
         if (valid) window_bounds(i, p.S, p.W, &w0, &nc);
+
+        // the block's Q rows -> shared memory (A operand: K-major, 128-byte
+        // swizzle), 16-byte units, all loads issued before the stores
+        {
+            constexpr int UPR = D / 8;
+            constexpr int NU = kRows * UPR / 128 / 2;     // two batches
+            const int tid = threadIdx.x - 64;
+#pragma unroll 1
+            for (int bt = 0; bt < 2; ++bt) {
+            uint4 v[NU];
+#pragma unroll
+            for (int q = 0; q < NU; ++q) {
+                const int e = tid + (bt * NU + q) * 128;
+                const int rr = e / UPR, u = e % UPR;
+                const int mi = i0 + rr / p.G;
+                v[q] = make_uint4(0u, 0u, 0u, 0u);
+                if (mi < p.N) {
+                    const int hq = p.group_heads[g * p.G + rr % p.G];
+                    v[q] = __ldg(reinterpret_cast<const uint4 *>(
+                               reinterpret_cast<const __nv_bfloat16 *>(p.Q) +
+                               (((int64_t)b * p.Hq + hq) * p.N + mi) * D) + u);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < NU; ++q) {
+                const int e = tid + (bt * NU + q) * 128;
+                const int rr = e / UPR, u = e % UPR;
+                *reinterpret_cast<uint4 *>(smem + L::OFF_Q + (u >> 3) * (kRows * 128) +
+                                           rr * 128 + (((u & 7) ^ (rr & 7)) << 4)) = v[q];
+            }
+            }
+            fence_async_smem();
+            mbar_arrive(&st.q_full);
+        }
+
         const int *myidx = s_idx + m;                    // stride M
         const int M_ = p.M;
         const float *mysel = p.sel + (((int64_t)b * p.Hq + h) * p.N + i) * p.K;
@@ -301,24 +331,19 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
         // s^ of the next selected chunk, loaded ahead of its tile
         float sh_next = (valid && p.K > 0) ? __ldg(mysel) : 0.f;
         const float sl2 = p.inv_sqrt_d * kLog2e;
+        const float2 sl2v = make_float2(sl2, sl2);
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
         bool ok = true;
 
         for (int t = 0; t < T; ++t) {
             const int sb = t & 1;
+            const uint32_t tS = trow + L::TMEM_S + sb * S_TOK;
             // every lane takes the same branch around warp-collective
             // tcgen05.ld / st, so wait outcomes are agreed across the warp
             if (!__all_sync(0xffffffffu, mbar_wait(&st.s_full[sb], (t >> 1) & 1, abort))) { ok = false; break; }
             tc_fence_after();
-            float x[S_TOK];
-#pragma unroll
-            for (int c0 = 0; c0 < S_TOK; c0 += 32) {
-                uint32_t rr[32];
-                tmem_ld32(trow + L::TMEM_S + sb * S_TOK + c0, rr);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 32; ++j) x[c0 + j] = __uint_as_float(rr[j]) * sl2;
-            }
+            uint32_t pk[S_TOK / 2];                      // P, bf16 pairs
+            float2 ps = make_float2(0.f, 0.f);           // sum of the rounded P
 
             if (t < U) {
                 const int c = s_union[t];
@@ -329,33 +354,70 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
                     sh_next = (valid && kp < p.K) ? __ldg(mysel + kp) : 0.f;
                 }
                 const bool sel = valid && kp < p.K && ck == c;
+                float sh = 0.f;
                 if (sel) {
-                    const float sh = sh_next * kLog2e;
+                    sh = sh_next * kLog2e;
                     ++kp;
                     sh_next = (kp < p.K) ? __ldg(mysel + kp) : 0.f;
-                    float mc = x[0];
+                }
+                if (__any_sync(0xffffffffu, sel)) {
+                    uint32_t rr[S_TOK];
 #pragma unroll
-                    for (int j = 1; j < S_TOK; ++j) mc = fmaxf(mc, x[j]);
-                    float z = 0.f;
+                    for (int c0 = 0; c0 < S_TOK; c0 += 32) tmem_ld32(tS + c0, rr + c0);
+                    tmem_wait_ld();
+                    if (sel) {
+                        // intra-chunk softmax scaled by exp(s^_c - M0) / z_c
+                        float mx = __uint_as_float(rr[0]);
 #pragma unroll
-                    for (int j = 0; j < S_TOK; ++j) { x[j] = fast_exp2(x[j] - mc); z += x[j]; }
-                    const float f = fast_exp2(sh - M0l2) / z;
+                        for (int j = 1; j < S_TOK; ++j) mx = fmaxf(mx, __uint_as_float(rr[j]));
+                        const float2 nb = make_float2(-mx * sl2, -mx * sl2);
+                        float2 e[S_TOK / 2];
+                        float2 z2 = make_float2(0.f, 0.f);
 #pragma unroll
-                    for (int j = 0; j < S_TOK; ++j) x[j] *= f;
+                        for (int j = 0; j < S_TOK / 2; ++j) {
+                            e[j] = f2_fma(make_float2(__uint_as_float(rr[2 * j]),
+                                                      __uint_as_float(rr[2 * j + 1])), sl2v, nb);
+                            e[j].x = fast_exp2(e[j].x);
+                            e[j].y = fast_exp2(e[j].y);
+                            z2 = f2_add(z2, e[j]);
+                        }
+                        const float f = fast_exp2(sh - M0l2) / (z2.x + z2.y);
+                        const float2 fv = make_float2(f, f);
+#pragma unroll
+                        for (int j = 0; j < S_TOK / 2; ++j) {
+                            const float2 pv = f2_mul(e[j], fv);
+                            pk[j] = pack_bf16(pv.x, pv.y);
+                            ps = f2_add(ps, make_float2(__uint_as_float(pk[j] << 16),
+                                                        __uint_as_float(pk[j] & 0xffff0000u)));
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < S_TOK / 2; ++j) pk[j] = 0u;
+                    }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < S_TOK; ++j) x[j] = 0.f;
+                    for (int j = 0; j < S_TOK / 2; ++j) pk[j] = 0u;
                 }
             } else {
                 const int j0 = wstart + (t - U) * S_TOK;
-                float mx = -INFINITY;
+                uint32_t rr[S_TOK];
 #pragma unroll
-                for (int j = 0; j < S_TOK; ++j) {
-                    const int pos = j0 + j;
-                    const bool in = valid && pos >= w0 && pos <= i;
-                    x[j] = in ? x[j] : -INFINITY;
-                    mx = fmaxf(mx, x[j]);
+                for (int c0 = 0; c0 < S_TOK; c0 += 32) tmem_ld32(tS + c0, rr + c0);
+                tmem_wait_ld();
+                // masks only where a row's window starts or ends in the tile
+                const bool edge = !valid || j0 < w0 || j0 + S_TOK - 1 > i;
+                if (__any_sync(0xffffffffu, edge)) {
+#pragma unroll
+                    for (int j = 0; j < S_TOK; ++j) {
+                        const int pos = j0 + j;
+                        const bool in = valid && pos >= w0 && pos <= i;
+                        rr[j] = in ? rr[j] : __float_as_uint(-INFINITY);
+                    }
                 }
+                float mx = __uint_as_float(rr[0]);
+#pragma unroll
+                for (int j = 1; j < S_TOK; ++j) mx = fmaxf(mx, __uint_as_float(rr[j]));
+                mx *= sl2;                                   // log2 units
                 const bool mine = mx > mref + kRescaleLog2;
                 if (__any_sync(0xffffffffu, mine)) {
                     // raise the reference max of the rows that need it and
@@ -368,22 +430,33 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
                         if (!__all_sync(0xffffffffu, mbar_wait(&st.p_empty[u & 1], (u >> 1) & 1, abort))) { ok = false; break; }
                         tc_fence_after();
 #pragma unroll
-                        for (int c0 = 0; c0 < D; c0 += 32) {
-                            uint32_t rr[32];
-                            tmem_ld32(trow + L::TMEM_O + c0, rr);
+                        for (int c0 = 0; c0 < D; c0 += 16) {
+                            uint32_t ro[16];
+                            tmem_ld16(trow + L::TMEM_O + c0, ro);
                             tmem_wait_ld();
 #pragma unroll
-                            for (int j = 0; j < 32; ++j)
-                                rr[j] = __float_as_uint(__uint_as_float(rr[j]) * fac);
-                            tmem_st32(trow + L::TMEM_O + c0, rr);
+                            for (int j = 0; j < 16; ++j)
+                                ro[j] = __float_as_uint(__uint_as_float(ro[j]) * fac);
+                            tmem_st16(trow + L::TMEM_O + c0, ro);
                         }
                         tmem_wait_st();
                     }
                     if (mine) { l *= fac; mref = mx; }
                 }
+                // rows with nothing in the window yet keep mref = -inf:
+                // their masked scores still give exp2(-inf) = 0
+                const float nm = (mref == -INFINITY) ? 0.f : -mref;
+                const float2 nmv = make_float2(nm, nm);
 #pragma unroll
-                for (int j = 0; j < S_TOK; ++j)
-                    x[j] = (x[j] == -INFINITY) ? 0.f : fast_exp2(x[j] - mref);
+                for (int j = 0; j < S_TOK / 2; ++j) {
+                    float2 e = f2_fma(make_float2(__uint_as_float(rr[2 * j]),
+                                                  __uint_as_float(rr[2 * j + 1])), sl2v, nmv);
+                    e.x = fast_exp2(e.x);
+                    e.y = fast_exp2(e.y);
+                    pk[j] = pack_bf16(e.x, e.y);
+                    ps = f2_add(ps, make_float2(__uint_as_float(pk[j] << 16),
+                                                __uint_as_float(pk[j] & 0xffff0000u)));
+                }
             }
 
             // P -> TMEM over this tile's S columns (bf16 pairs), then the MMA.
@@ -391,18 +464,9 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
             // the weights applied to V add up to one: in a peaked row the
             // rounding of P then moves O by ~2^-9 w(1-w)|v| instead of
             // ~2^-9 w|v|.
-            float ps = 0.f;
 #pragma unroll
-            for (int c0 = 0; c0 < S_TOK; c0 += 64) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    pk[j] = pack_bf16(x[c0 + 2 * j], x[c0 + 2 * j + 1]);
-                    ps += __uint_as_float(pk[j] << 16) + __uint_as_float(pk[j] & 0xffff0000u);
-                }
-                tmem_st32(trow + L::TMEM_S + sb * S_TOK + c0 / 2, pk);
-            }
-            l += ps;
+            for (int c0 = 0; c0 < S_TOK / 2; c0 += 32) tmem_st32(tS + c0, pk + c0);
+            l += ps.x + ps.y;
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&st.p_full[sb]);
@@ -420,17 +484,17 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmQ,
                                   (((int64_t)b * p.Hq + h) * p.N + i) * D;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t rr[32];
-                tmem_ld32(trow + L::TMEM_O + c0, rr);
+                uint32_t ro[32];
+                tmem_ld32(trow + L::TMEM_O + c0, ro);
                 tmem_wait_ld();
                 if (valid) {
 #pragma unroll
                     for (int j = 0; j < 32; j += 8) {
                         uint4 v;
-                        v.x = pack_bf16(__uint_as_float(rr[j + 0]) * inv, __uint_as_float(rr[j + 1]) * inv);
-                        v.y = pack_bf16(__uint_as_float(rr[j + 2]) * inv, __uint_as_float(rr[j + 3]) * inv);
-                        v.z = pack_bf16(__uint_as_float(rr[j + 4]) * inv, __uint_as_float(rr[j + 5]) * inv);
-                        v.w = pack_bf16(__uint_as_float(rr[j + 6]) * inv, __uint_as_float(rr[j + 7]) * inv);
+                        v.x = pack_bf16(__uint_as_float(ro[j + 0]) * inv, __uint_as_float(ro[j + 1]) * inv);
+                        v.y = pack_bf16(__uint_as_float(ro[j + 2]) * inv, __uint_as_float(ro[j + 3]) * inv);
+                        v.z = pack_bf16(__uint_as_float(ro[j + 4]) * inv, __uint_as_float(ro[j + 5]) * inv);
+                        v.w = pack_bf16(__uint_as_float(ro[j + 6]) * inv, __uint_as_float(ro[j + 7]) * inv);
                         *reinterpret_cast<uint4 *>(orow + c0 + j) = v;
                     }
                 }
@@ -464,7 +528,7 @@ cudaError_t launch_attend_t(const TcParams &tp, const TcMaps &maps,
     const int nqb = (tp.N + tp.M - 1) / tp.M;
     const int64_t grid = (int64_t)tp.B * tp.Hkv * nqb;
     if (grid <= 0) return cudaSuccess;
-    kern<<<(unsigned)grid, kThreads, smem, st>>>(maps.q, maps.k, maps.v, tp);
+    kern<<<(unsigned)grid, kThreads, smem, st>>>(maps.k, maps.v, tp);
     (void)sizeof(L);
     return cudaGetLastError();
 }

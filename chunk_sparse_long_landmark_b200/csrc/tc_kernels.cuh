@@ -9,6 +9,7 @@
 namespace hils {
 
 struct TcParams {
+    const void *Q;  // [B,Hq,N,d] (the attention kernel loads its rows itself)
     const void *Klm;
     const float *bias;
     void *O;
@@ -23,7 +24,6 @@ struct TcParams {
 };
 
 struct TcMaps {
-    CUtensorMap q;  // Q or Qs [B,Hq,N,d]: box {64, M, 1, 1}
     CUtensorMap k;  // K [B,Hkv,N,d]: box {64, S, 1, 1}
     CUtensorMap v;  // V [B,Hkv,N,d]: box {64, S, 1, 1}
     CUtensorMap lm; // Klm [B,Hkv,nC,d]: box {64, 128, 1, 1}

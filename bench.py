@@ -302,6 +302,52 @@ def workload_config(sh, name):
                            "(batch, kv head), no collective)"}
 
 
+# ------------------------------------------------------------ rank plumbing
+class RankContext:
+    """One process per GPU, launched by torchrun (RANK / WORLD_SIZE / MASTER_*
+    from the environment). Each rank runs its own replica of the workload
+    (the path shards by (batch, kv head) with no exchange), so the only
+    collectives are the barrier around the timed region and the max over
+    ranks of the measured time. `backend` is "nccl" on GPUs; the same code
+    runs on "gloo" with CPU tensors."""
+
+    def __init__(self, backend="nccl", device=None, timeout_s=300):
+        import torch
+        import torch.distributed as dist
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.device = device if device is not None else torch.device("cpu")
+        self._dist = None
+        if self.world > 1:
+            from datetime import timedelta
+            kw = {"device_id": self.device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=timedelta(seconds=timeout_s),
+                                    **kw)
+            self._dist = dist
+
+    def barrier(self):
+        if self._dist is not None:
+            self._dist.barrier()
+
+    def max(self, x):
+        """Largest value of x over all ranks (a device-timed duration)."""
+        import torch
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
+        if self._dist is not None:
+            self._dist.all_reduce(t, op=self._dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def whole_job_rate(self, units_per_rank, ms_max):
+        """Units all ranks processed per second, over the slowest rank's
+        time (ms_max, already the max over ranks)."""
+        return self.world * units_per_rank / (ms_max * 1e-3)
+
+    def close(self):
+        if self._dist is not None:
+            self._dist.destroy_process_group()
+            self._dist = None
+
+
 # ---------------------------------------------------------------- GPU arm
 def main():
     ap = argparse.ArgumentParser()
@@ -327,30 +373,15 @@ def main():
         return
 
     import torch
-    import torch.distributed as dist
 
     import chunk_sparse_long_landmark_b200 as hils
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        from datetime import timedelta
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = RankContext("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     peaks = measured_peaks()
     if args.decode_only:
@@ -359,8 +390,7 @@ def main():
                          world, max_over_ranks, barrier, rank, peaks)
         if rank == 0:
             print(json.dumps({"decode": d}), flush=True)
-        if world > 1:
-            dist.destroy_process_group()
+        ranks.close()
         return
     inp = synth.make_prefill(sh, seed=synth.seed_for(cfg_id) + 17 * rank,
                              device=dev)
@@ -408,7 +438,7 @@ def main():
     t_step = [a + b for a, b in zip(t_sel, t_att)]
     tot_ms = max_over_ranks(sum(t_step))
     ms_step = tot_ms / args.steps
-    value = world * work["tokens"] / (ms_step * 1e-3)
+    value = ranks.whole_job_rate(work["tokens"], ms_step)
 
     # dominant kernel roofline (tensor-bound contraction)
     a_ms, s_ms = statistics.mean(t_att), statistics.mean(t_sel)
@@ -499,8 +529,7 @@ def main():
 
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    ranks.close()
 
 
 def bench_decode(args, dev, stream, flush, world, max_over_ranks, barrier,

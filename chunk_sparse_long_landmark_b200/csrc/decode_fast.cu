@@ -14,12 +14,13 @@
 //               group score a_c = max_h (s^_hc - LSE_h), exact top-K by a
 //               4-round radix select (ties to the lower chunk), idx
 //               ascending, s^ of the selected chunks.
-//   dec_attend  one CTA per (b, kv head, selected chunk or window tile):
-//               K/V tile by TMA, QK^T and PV with mma.sync, intra-chunk
-//               softmax scaled by exp(s^_c) (chunk tiles) or plain masked
-//               softmax (window tiles) -> partial (m, l, o); the CTA that
-//               arrives last for its (b, kv head) combines the partials in
-//               tile order (deterministic) and writes O.
+//   dec_attend  one CTA per (b, kv head, group of selected-chunk / window
+//               tiles), one wave in all: K/V tiles double-buffered by TMA,
+//               QK^T and PV with mma.sync, intra-chunk softmax scaled by
+//               exp(s^_c) (chunk tiles) or plain masked softmax (window
+//               tiles), merged online -> partial (m, l, o) per group; the
+//               CTA that arrives last for its (b, kv head) combines the
+//               partials in group order (deterministic) and writes O.
 #include <math.h>
 
 #include "hils_fast.cuh"

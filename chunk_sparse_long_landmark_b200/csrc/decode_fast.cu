@@ -293,6 +293,8 @@ __device__ int block_excl_scan(int v, int *scratch, int *total) {
 }
 
 constexpr int kSelPer = 16;                      // chunks per thread (<= 16384)
+constexpr int kCandCap = 1024;                   // threshold-path candidate list
+constexpr int kMaxSplits = 64;                   // staged landmark-split partials
 
 __global__ void __launch_bounds__(kSelThreads)
 dec_select_kernel(const DecParams p) {
@@ -300,6 +302,12 @@ dec_select_kernel(const DecParams p) {
     __shared__ int hist[256];
     __shared__ int scan_scr[33];
     __shared__ int sh_digit, sh_need;
+    __shared__ float part[kMaxSplits * 8][2];
+    __shared__ uint32_t wtop[2 * (kSelThreads / 32)];
+    __shared__ uint32_t sh_tau;
+    __shared__ int ncand;
+    __shared__ uint32_t cand_k[kCandCap];
+    __shared__ int cand_c[kCandCap];
     const int g = blockIdx.x, b = blockIdx.y;
     const int bg = b * p.Hkv + g;
     const int G = p.G, K = p.K;
@@ -308,12 +316,22 @@ dec_select_kernel(const DecParams p) {
     const int nc = (int)nc64;
     const float *ss = p.ws_s + (int64_t)bg * G * p.ncs;
 
-    if (threadIdx.x < G) {                       // merge the split partials
+    // merge the split partials: all loaded at once into shared memory, then
+    // folded in split order by one thread per head
+    const int nsp = (nc + p.cps - 1) / p.cps;
+    const bool staged = nsp * G <= kSelThreads && nsp <= kMaxSplits;
+    if (staged && threadIdx.x < nsp * G) {
+        const float *pp = p.ws_p + ((int64_t)bg * p.nsplit * G + threadIdx.x) * 2;
+        part[threadIdx.x][0] = pp[0];
+        part[threadIdx.x][1] = pp[1];
+    }
+    __syncthreads();
+    if (threadIdx.x < G) {
         const int hh = threadIdx.x;
         float m = -INFINITY, s2 = 0.f;
-        const int nsp = (nc + p.cps - 1) / p.cps;
         for (int sp = 0; sp < nsp; ++sp) {
-            const float *pp = p.ws_p + (((int64_t)bg * p.nsplit + sp) * G + hh) * 2;
+            const float *pp = staged ? part[sp * G + hh]
+                                     : p.ws_p + (((int64_t)bg * p.nsplit + sp) * G + hh) * 2;
             const float om = pp[0], os = pp[1];
             const float mn = fmaxf(m, om);
             s2 = (mn == -INFINITY) ? 0.f : s2 * exp2f(m - mn) + os * exp2f(om - mn);
@@ -324,21 +342,117 @@ dec_select_kernel(const DecParams p) {
     __syncthreads();
 
     // group scores of this thread's contiguous chunks c = tid * per + q
-    const int per = (nc + kSelThreads - 1) / kSelThreads;   // <= kSelPer
+    // a multiple of 4 (16-byte loads), at most kSelPer
+    const int per = ((nc + kSelThreads - 1) / kSelThreads + 3) & ~3;
     const int cbeg = threadIdx.x * per;
+    // head by head, the thread's chunks loaded together (one round trip
+    // per head instead of one per chunk and head)
+    float amax[kSelPer];
+#pragma unroll
+    for (int q = 0; q < kSelPer; ++q) amax[q] = -INFINITY;
+    for (int hh = 0; hh < G; ++hh) {
+        const float *row = ss + (int64_t)hh * p.ncs;
+        const float lh = lse[hh];
+        float v[kSelPer];
+#pragma unroll
+        for (int q4 = 0; q4 < kSelPer / 4; ++q4) {
+            // rows are padded to a multiple of 4: values past nc are read
+            // but never turned into keys
+            float4 f = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            if (4 * q4 < per && cbeg + 4 * q4 < nc)
+                f = __ldcg(reinterpret_cast<const float4 *>(row + cbeg + 4 * q4));
+            v[4 * q4 + 0] = f.x; v[4 * q4 + 1] = f.y;
+            v[4 * q4 + 2] = f.z; v[4 * q4 + 3] = f.w;
+        }
+#pragma unroll
+        for (int q = 0; q < kSelPer; ++q) amax[q] = fmaxf(amax[q], v[q] - lh);
+    }
     uint32_t key[kSelPer];
 #pragma unroll
-    for (int q = 0; q < kSelPer; ++q) {
-        const int c = cbeg + q;
-        key[q] = 0u;                             // below every real key
-        if (q < per && c < nc) {
-            float a = -INFINITY;
-            for (int hh = 0; hh < G; ++hh)
-                a = fmaxf(a, ss[(int64_t)hh * p.ncs + c] - lse[hh]);
-            key[q] = order_key(a);
+    for (int q = 0; q < kSelPer; ++q)                // 0: below every real key
+        key[q] = (q < per && cbeg + q < nc) ? order_key(amax[q]) : 0u;
+    const int nsel = min(nc, K);
+
+    // Threshold path. Each warp's two largest keys belong to distinct
+    // chunks, so the K-th largest of those 2 x 32 values is a lower bound on
+    // the K-th largest key (K <= 64). Only keys at or above it become
+    // candidates; their exact ranks (ties: lower chunk first) are counted
+    // over the short list. A list longer than kCandCap (exact or near ties
+    // over many chunks) falls through to the radix select below.
+    if (nc > K && K <= 2 * (kSelThreads / 32)) {
+        uint32_t t1 = 0u, t2 = 0u;               // this thread's two largest
+#pragma unroll
+        for (int q = 0; q < kSelPer; ++q) {
+            const uint32_t k = key[q];
+            t2 = max(t2, min(t1, k));
+            t1 = max(t1, k);
+        }
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+        for (int o = 1; o < 32; o <<= 1) {       // warp top-2 (merge of pairs)
+            const uint32_t o1 = __shfl_xor_sync(0xffffffffu, t1, o);
+            const uint32_t o2 = __shfl_xor_sync(0xffffffffu, t2, o);
+            const uint32_t n1 = max(t1, o1);
+            t2 = max(min(t1, o1), max(t2, o2));
+            t1 = n1;
+        }
+        if (lane == 0) { wtop[2 * warp] = t1; wtop[2 * warp + 1] = t2; }
+        if (threadIdx.x == 0) ncand = 0;
+        __syncthreads();
+        if (warp == 0) {
+            // largest v among the 64 with at least K of them >= v
+            uint32_t best = 0u;
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2) {
+                const uint32_t v = wtop[2 * lane + s2];
+                int ge = 0;
+                for (int f = 0; f < 2 * (kSelThreads / 32); ++f) ge += (wtop[f] >= v) ? 1 : 0;
+                if (ge >= K) best = max(best, v);
+            }
+            for (int o = 1; o < 32; o <<= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+            if (lane == 0) sh_tau = best;
+        }
+        __syncthreads();
+        const uint32_t tau = sh_tau;
+#pragma unroll
+        for (int q = 0; q < kSelPer; ++q) {
+            const int c = cbeg + q;
+            if (q < per && c < nc && key[q] >= tau) {
+                const int at = atomicAdd(&ncand, 1);
+                if (at < kCandCap) { cand_k[at] = key[q]; cand_c[at] = c; }
+            }
+        }
+        __syncthreads();
+        const int m = ncand;
+        if (m <= kCandCap) {
+            bool mine = false;
+            uint32_t mk = 0u;
+            int mc = 0;
+            if (threadIdx.x < m) {
+                mk = cand_k[threadIdx.x];
+                mc = cand_c[threadIdx.x];
+                int rank = 0;
+                for (int f = 0; f < m; ++f) {
+                    const uint32_t fk = cand_k[f];
+                    rank += (fk > mk || (fk == mk && cand_c[f] < mc)) ? 1 : 0;
+                }
+                mine = rank < K;
+            }
+            __syncthreads();                     // ranks read the list first
+            if (threadIdx.x < m) cand_k[threadIdx.x] = mine ? 1u : 0u;
+            __syncthreads();
+            if (mine) {                          // ascending chunk order
+                int pos = 0;
+                for (int f = 0; f < m; ++f) pos += (cand_k[f] && cand_c[f] < mc) ? 1 : 0;
+                p.idx[(int64_t)bg * K + pos] = mc;
+                for (int hh = 0; hh < G; ++hh) {
+                    const int h = p.group_heads[g * G + hh];
+                    p.sel[((int64_t)b * p.Hq + h) * K + pos] = ss[(int64_t)hh * p.ncs + mc];
+                }
+            }
+            return;                              // nc > K: no padding
         }
     }
-    const int nsel = min(nc, K);
+
     uint32_t thr = 0u;                           // selected: key > thr, or == thr and early
     int need_eq = 0;
     if (nc > K) {
@@ -450,8 +564,13 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     __shared__ uint64_t bar[2];
     __shared__ float red[4][8];
+    __shared__ float rmx[2][4][8], rsm[2][4][8];
     __shared__ int last;
-    float *ored = reinterpret_cast<float *>(smem + 4 * TB);     // [4][8][D]
+    __shared__ int s_idx[HILS_MAX_TOPK];
+    __shared__ float s_sel[8 * HILS_MAX_TOPK];   // G <= 8 on this path
+    // [4][8][D] partial O of the 4 warps: used only after the tile loop, when
+    // every copy has landed and been read, so it shares the stage buffers
+    float *ored = reinterpret_cast<float *>(smem);
 
     const int grp = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int bg = b * p.Hkv + g;
@@ -460,16 +579,25 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     const int G = p.G;
     int64_t i = 0, w0 = 0, nc = 0;
     const bool ok = seq_ok(p, b, &i, &w0, &nc);
+    // this (b, g)'s selection -- chunk indices and the heads' s^ -- staged
+    // once, so no tile waits on a global load for them
+    for (int e = threadIdx.x; e < p.K; e += kAttThreads)
+        s_idx[e] = ok ? p.idx[(int64_t)bg * p.K + e] : -1;
+    for (int e = threadIdx.x; e < G * p.K; e += kAttThreads) {
+        const int hh = e / p.K, kk = e % p.K;
+        const int h = p.group_heads[g * G + hh];
+        s_sel[e] = ok ? p.sel[((int64_t)b * p.Hq + h) * p.K + kk] : 0.f;
+    }
+    __syncthreads();
     int nsel = 0;
-    if (ok)
-        for (int k = 0; k < p.K; ++k) nsel += (p.idx[(int64_t)bg * p.K + k] >= 0) ? 1 : 0;
+    for (int k = 0; k < p.K; ++k) nsel += (s_idx[k] >= 0) ? 1 : 0;
     const int nwin = ok ? (int)((i - w0 + 1 + S_TOK - 1) / S_TOK) : 0;
     const int ntot = nsel + nwin;
     const int tb = grp * p.att_per;
     const int te = min(tb + p.att_per, ntot);
     const int nmine = te > tb ? te - tb : 0;
     auto tile_j0 = [&](int tau) -> int64_t {
-        return tau < nsel ? (int64_t)p.idx[(int64_t)bg * p.K + tau] * p.S
+        return tau < nsel ? (int64_t)s_idx[tau] * p.S
                           : w0 + (int64_t)(tau - nsel) * S_TOK;
     };
     volatile int dummy_abort = 0;
@@ -540,6 +668,10 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                     mma_bf16(sacc[np2 + 1], aq[ks], bm[2], bm[3]);
                 }
             }
+            // row max and sum: each warp over its tokens (relative to its
+            // own max), then one exchange; the arrays alternate with the
+            // tile parity, so the next tile's writes never meet this tile's
+            // reads (all threads pass the next top barrier first)
             float mloc = -INFINITY;
 #pragma unroll
             for (int n = 0; n < NT; ++n)
@@ -553,31 +685,35 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                 }
             mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
             mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-            if (t == 0) red[warp][gi] = mloc;
-            __syncthreads();
-            const float m = fmaxf(fmaxf(red[0][gi], red[1][gi]), fmaxf(red[2][gi], red[3][gi]));
-            __syncthreads();
             float sloc = 0.f;
 #pragma unroll
             for (int n = 0; n < NT; ++n)
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
-                    const float e = (sacc[n][q] == -INFINITY) ? 0.f : fast_exp2(sacc[n][q] - m);
+                    const float e = (sacc[n][q] == -INFINITY) ? 0.f : fast_exp2(sacc[n][q] - mloc);
                     sacc[n][q] = e;
                     sloc += e;
                 }
             sloc += __shfl_xor_sync(0xffffffffu, sloc, 1);
             sloc += __shfl_xor_sync(0xffffffffu, sloc, 2);
-            if (t == 0) red[warp][gi] = sloc;
+            if (t == 0) { rmx[k & 1][warp][gi] = mloc; rsm[k & 1][warp][gi] = sloc; }
             __syncthreads();
-            const float z = red[0][gi] + red[1][gi] + red[2][gi] + red[3][gi];
-            __syncthreads();
+            float m = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) m = fmaxf(m, rmx[k & 1][w][gi]);
+            float z = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float mw = rmx[k & 1][w][gi];
+                z += (mw == -INFINITY) ? 0.f : rsm[k & 1][w][gi] * fast_exp2(mw - m);
+            }
+            // this warp's values are relative to mloc: bring them to m
+            const float fw = (mloc == -INFINITY) ? 0.f : fast_exp2(mloc - m);
             // this tile's weights relative to its own reference m_t:
             // chunk tile: m_t = s^_c, weights e/z; window: m_t = max, weights e
             float m_t, scale_t;
             if (is_chunk) {
-                const int h = (gi < G) ? p.group_heads[g * G + gi] : 0;
-                m_t = (gi < G) ? p.sel[((int64_t)b * p.Hq + h) * p.K + tau] : 0.f;
+                m_t = (gi < G) ? s_sel[gi * p.K + tau] : 0.f;
                 scale_t = 1.f / z;
             } else {
                 m_t = m / kLog2e;
@@ -594,7 +730,7 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
             Mrun = Mn;
 #pragma unroll
             for (int n = 0; n < D / 8; ++n) { oacc[n][0] *= fo; oacc[n][1] *= fo; }
-            const float ws = scale_t * fn;
+            const float ws = scale_t * fn * fw;
 #pragma unroll
             for (int kk = 0; kk < TOK_W / 16; ++kk) {
                 uint32_t ap[4];
@@ -666,21 +802,43 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     if (!last || !ok) return;
     __threadfence();
     const int ngrp = (ntot + p.att_per - 1) / p.att_per;
+    // per group and head: w_gg / sum_gg' w_gg' l_gg' with w = exp(m - max m)
+    // (the stage buffers are free now), then O = sum of weighted partial O
+    // in group order, the partial loads of 8 groups issued together
+    float *cw = reinterpret_cast<float *>(smem);             // [ngrp][G]
+    if (threadIdx.x < G) {
+        const int hh = threadIdx.x;
+        const float *mlb = p.ws_ml + ((int64_t)bg * p.ntile * G + hh) * 2;
+        float M = -INFINITY;
+#pragma unroll 8
+        for (int gg = 0; gg < ngrp; ++gg) M = fmaxf(M, __ldcg(mlb + (int64_t)gg * G * 2));
+        float den = 0.f;
+#pragma unroll 8
+        for (int gg = 0; gg < ngrp; ++gg) {
+            const float w = exp2f((__ldcg(mlb + (int64_t)gg * G * 2) - M) * kLog2e);
+            cw[gg * G + hh] = w;
+            den += w * __ldcg(mlb + (int64_t)gg * G * 2 + 1);
+        }
+        const float inv = 1.f / den;
+        for (int gg = 0; gg < ngrp; ++gg) cw[gg * G + hh] *= inv;
+    }
+    __syncthreads();
     for (int e = threadIdx.x; e < G * D; e += kAttThreads) {
         const int hh = e / D, c = e % D;
-        float M = -INFINITY;
-        for (int gg = 0; gg < ngrp; ++gg)
-            M = fmaxf(M, __ldcg(p.ws_ml + (((int64_t)bg * p.ntile + gg) * G + hh) * 2));
-        float num = 0.f, den = 0.f;
-        for (int gg = 0; gg < ngrp; ++gg) {
-            const float *ml = p.ws_ml + (((int64_t)bg * p.ntile + gg) * G + hh) * 2;
-            const float w = exp2f((__ldcg(ml) - M) * kLog2e);
-            den += w * __ldcg(ml + 1);
-            num += w * __ldcg(p.ws_o + (((int64_t)bg * p.ntile + gg) * G + hh) * D + c);
+        const float *ob = p.ws_o + ((int64_t)bg * p.ntile * G + hh) * D + c;
+        float num = 0.f;
+        for (int g0 = 0; g0 < ngrp; g0 += 8) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                v[u] = (g0 + u < ngrp) ? __ldcg(ob + (int64_t)(g0 + u) * G * D) : 0.f;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (g0 + u < ngrp) num += cw[(g0 + u) * G + hh] * v[u];
         }
         const int h = p.group_heads[g * G + hh];
         reinterpret_cast<__nv_bfloat16 *>(p.O)[((int64_t)b * p.Hq + h) * D + c] =
-            __float2bfloat16_rn(num / den);
+            __float2bfloat16_rn(num);
     }
     if (threadIdx.x == 0) p.ws_cnt[bg] = 0;      // ready for the next call
 }
@@ -718,7 +876,8 @@ DecPlan dec_plan(const Problem &p) {
     DecPlan pl;
     int64_t w0, ncm;
     window_bounds((int64_t)p.kv_rows - 1, p.S, p.W, &w0, &ncm);
-    pl.ncs = (int)(ncm > 0 ? ncm : 1);
+    // s^ rows padded to a multiple of 4 floats: 16-byte loads in dec_select
+    pl.ncs = (int)(((ncm > 0 ? ncm : 1) + 3) & ~(int64_t)3);
     // splits sized so that about 3 CTAs per SM stream the whole scan
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
@@ -733,7 +892,8 @@ DecPlan dec_plan(const Problem &p) {
     pl.cps = (int)(tps * kTileChunks);
     pl.nsplit = (pl.ncs + pl.cps - 1) / pl.cps;
     pl.ntile = p.K + (p.W + 2 * p.S - 2) / p.S + 1;
-    // attention: one wave of CTAs (2 resident per SM at S = 64, 1 at S = 128)
+    // attention: one wave of CTAs, 2 per SM at S = 64 (measured faster than
+    // 3 shorter ones), 1 at S = 128
     {
         const int64_t slots = (int64_t)sms * (p.S == 64 ? 2 : 1);
         int64_t groups = slots / ((int64_t)p.B * p.Hkv);
@@ -818,7 +978,8 @@ cudaError_t launch_dec_select(Problem &p, void *ws, cudaStream_t st) {
 template <int S_TOK, int D>
 cudaError_t launch_att_t(const DecParams &d, const CUtensorMap &tk,
                          const CUtensorMap &tv, cudaStream_t st) {
-    const size_t smem = 1024 + 4ull * S_TOK * D * 2 + 4ull * 8 * D * 4;
+    static_assert(4 * 8 * D * 4 <= 4 * S_TOK * D * 2, "partial O fits the stages");
+    const size_t smem = 1024 + 4ull * S_TOK * D * 2;
     cudaError_t e = cudaFuncSetAttribute(dec_attend_kernel<S_TOK, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);

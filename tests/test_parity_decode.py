@@ -102,3 +102,31 @@ def test_decode_deterministic_and_graph(cuda_device):
     torch.cuda.synchronize()
     assert torch.equal(O, O1) and torch.equal(idx, i1)
     del g
+
+
+@pytest.mark.parametrize("every", [80, 2])
+def test_decode_exact_score_ties_take_lower_chunks(every, cuda_device):
+    """Identical landmark keys; b' = 0 on chunks c % every == 0, -1 elsewhere.
+    The tied chunks share one group score exactly, so the tie rule alone
+    decides: idx must be the K lowest tied chunks of C_i, bit for bit.
+    every=80 gives ~100 tied chunks (a short candidate list); every=2 ties
+    half of all candidates (too many for a short list)."""
+    sh = synth.Shape("bf16", 2, 32, 8, 128, 16384, 64, 512, 32)
+    lens = [16384, 9000]
+    inp = synth.make_decode(sh, seed=211, device=cuda_device, cache_len=lens)
+    nC = sh.N // sh.S
+    klm = inp["Klm"][:, :, :1, :].expand(-1, -1, nC, -1).contiguous()
+    bias = torch.full((sh.B, sh.Hkv, nC), -1.0, dtype=torch.float32,
+                      device=cuda_device)
+    bias[:, :, 0::every] = 0.0
+    inp = dict(inp, Klm=klm, bias=bias)
+    O, idx = run_decode(inp)
+    got = idx.cpu().numpy()
+    for b, L in enumerate(lens):
+        nc = max((L - 1 - sh.W + 1) // sh.S, 0)
+        c = np.arange(nc)
+        order = np.concatenate([c[c % every == 0], c[c % every != 0]])[:sh.K]
+        want = np.sort(order)
+        for g in range(sh.Hkv):
+            np.testing.assert_array_equal(got[b, g], want)
+    parity.check_decode(inp, O, idx)

@@ -217,6 +217,7 @@ dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
         }
     }
     (void)sl2;
+    grid_dep_launch();                           // dec_select may start now
     if (dummy_abort) {                           // a tile never arrived
         if (threadIdx.x == 0) {
             report(p.status, HILS_ERR_DEVICE_TIMEOUT);
@@ -315,6 +316,8 @@ dec_select_kernel(const DecParams p) {
     if (!seq_ok(p, b, &i, &w0, &nc64)) return;
     const int nc = (int)nc64;
     const float *ss = p.ws_s + (int64_t)bg * G * p.ncs;
+    grid_dep_wait();                             // dec_score's s^ and partials
+    grid_dep_launch();                           // dec_attend may start now
 
     // merge the split partials: all loaded at once into shared memory, then
     // folded in split order by one thread per head
@@ -579,18 +582,9 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     const int G = p.G;
     int64_t i = 0, w0 = 0, nc = 0;
     const bool ok = seq_ok(p, b, &i, &w0, &nc);
-    // this (b, g)'s selection -- chunk indices and the heads' s^ -- staged
-    // once, so no tile waits on a global load for them
-    for (int e = threadIdx.x; e < p.K; e += kAttThreads)
-        s_idx[e] = ok ? p.idx[(int64_t)bg * p.K + e] : -1;
-    for (int e = threadIdx.x; e < G * p.K; e += kAttThreads) {
-        const int hh = e / p.K, kk = e % p.K;
-        const int h = p.group_heads[g * G + hh];
-        s_sel[e] = ok ? p.sel[((int64_t)b * p.Hq + h) * p.K + kk] : 0.f;
-    }
-    __syncthreads();
-    int nsel = 0;
-    for (int k = 0; k < p.K; ++k) nsel += (s_idx[k] >= 0) ? 1 : 0;
+    // the selection always holds min(|C_i|, K) chunks, so the tile list is
+    // known before the selection itself is read
+    const int nsel = ok ? (int)min(nc, (int64_t)p.K) : 0;
     const int nwin = ok ? (int)((i - w0 + 1 + S_TOK - 1) / S_TOK) : 0;
     const int ntot = nsel + nwin;
     const int tb = grp * p.att_per;
@@ -603,26 +597,42 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     volatile int dummy_abort = 0;
     bool arrived_all = true;
 
+    if (threadIdx.x == 0 && nmine > 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    auto issue = [&](int k) {                    // tile tb + k into buffer k & 1
+        const int64_t row = (int64_t)bg * p.Lmax + tile_j0(tb + k);
+        uint8_t *dst = smem + (k & 1) * 2 * TB;
+        mbar_expect_tx(&bar[k & 1], 2 * TB);
+        for (int hf = 0; hf < HALVES; ++hf) {
+            tma_load_2d(dst + hf * (S_TOK * 128), &tmK, &bar[k & 1], hf * 64, (int)row);
+            tma_load_2d(dst + TB + hf * (S_TOK * 128), &tmV, &bar[k & 1], hf * 64, (int)row);
+        }
+    };
+    // window tiles need nothing from the selection: their copies start
+    // before the wait for the selection kernel
+    if (threadIdx.x == 0)
+        for (int k = 0; k < min(nmine, 2); ++k)
+            if (tb + k >= nsel) issue(k);
+    grid_dep_wait();                             // dec_select's idx and s^
+    // this (b, g)'s selection -- chunk indices and the heads' s^ -- staged
+    // once, so no tile waits on a global load for them
+    for (int e = threadIdx.x; e < p.K; e += kAttThreads)
+        s_idx[e] = ok ? p.idx[(int64_t)bg * p.K + e] : -1;
+    for (int e = threadIdx.x; e < G * p.K; e += kAttThreads) {
+        const int hh = e / p.K, kk = e % p.K;
+        const int h = p.group_heads[g * G + hh];
+        s_sel[e] = ok ? p.sel[((int64_t)b * p.Hq + h) * p.K + kk] : 0.f;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0)
+        for (int k = 0; k < min(nmine, 2); ++k)
+            if (tb + k < nsel) issue(k);
+
     if (nmine > 0) {
-        if (threadIdx.x == 0) {
-            mbar_init(&bar[0], 1);
-            mbar_init(&bar[1], 1);
-            fence_barrier_init();
-        }
-        __syncthreads();
-        auto issue = [&](int k) {                // tile tb + k into buffer k & 1
-            const int64_t row = (int64_t)bg * p.Lmax + tile_j0(tb + k);
-            uint8_t *dst = smem + (k & 1) * 2 * TB;
-            mbar_expect_tx(&bar[k & 1], 2 * TB);
-            for (int hf = 0; hf < HALVES; ++hf) {
-                tma_load_2d(dst + hf * (S_TOK * 128), &tmK, &bar[k & 1], hf * 64, (int)row);
-                tma_load_2d(dst + TB + hf * (S_TOK * 128), &tmV, &bar[k & 1], hf * 64, (int)row);
-            }
-        };
-        if (threadIdx.x == 0) {
-            issue(0);
-            if (nmine > 1) issue(1);
-        }
         // Q as the A operand: row = head slot gi (< G), cols = dims
         uint32_t aq[D / 16][4];
 #pragma unroll
@@ -935,6 +945,25 @@ DecParams dec_params(const Problem &p, void *ws) {
 
 }  // namespace
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// its predecessor finishes, and waits for it (grid_dep_wait) before reading
+// what it wrote.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block,
+                             size_t smem, cudaStream_t st, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 bool dec_fast_supported(const Problem &p) {
     if (!p.decode || p.dtype != HILS_BF16) return false;
     if (!(p.d == 64 || p.d == 128) || !(p.S == 64 || p.S == 128)) return false;
@@ -970,9 +999,9 @@ cudaError_t launch_dec_select(Problem &p, void *ws, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    dec_select_kernel<<<dim3(p.Hkv, p.B), kSelThreads, 0, st>>>(d);
+    e = launch_dependent(dec_select_kernel, dim3(p.Hkv, p.B), dim3(kSelThreads), 0, st, d);
     count_launches(2);
-    return cudaGetLastError();
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <int S_TOK, int D>
@@ -985,8 +1014,9 @@ cudaError_t launch_att_t(const DecParams &d, const CUtensorMap &tk,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const int ngrp = (d.ntile + d.att_per - 1) / d.att_per;
-    dec_attend_kernel<S_TOK, D><<<dim3(ngrp, d.Hkv, d.B), kAttThreads, smem, st>>>(tk, tv, d);
-    return cudaGetLastError();
+    e = launch_dependent(dec_attend_kernel<S_TOK, D>, dim3(ngrp, d.Hkv, d.B),
+                         dim3(kAttThreads), smem, st, tk, tv, d);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 cudaError_t launch_dec_attend(Problem &p, void *ws, cudaStream_t st) {

@@ -87,6 +87,20 @@ __device__ __forceinline__ bool mbar_drain(uint64_t *bar, uint32_t parity) {
     return true;
 }
 
+// ------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialisation may start while
+// its predecessor in the stream is still running. It must call
+// grid_dep_wait() before reading anything the predecessor writes: the wait
+// returns once that grid has completed and its memory is visible.
+// grid_dep_launch() lets the successor start early (a hint; without it the
+// successor starts when this grid completes).
+__device__ __forceinline__ void grid_dep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // -------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map,
                                             uint64_t *bar, int c0, int c1,

@@ -516,6 +516,8 @@ def main():
     if not args.no_decode:
         line["decode"] = bench_decode(args, dev, stream, flush, world,
                                       max_over_ranks, barrier, rank, peaks)
+        line["landmarks"] = bench_landmarks(args, dev, stream, flush,
+                                            max_over_ranks, barrier, peaks)
 
     if rank == 0 and world == 1 and not args.no_cpu:
         cinp = synth.make_prefill(sh, seed=synth.seed_for(cfg_id),
@@ -530,6 +532,54 @@ def main():
     if rank == 0:
         print(json.dumps(line), flush=True)
     ranks.close()
+
+
+def bench_landmarks(args, dev, stream, flush, max_over_ranks, barrier,
+                    peaks):
+    """Landmark summaries (Prop. 3.1) of the 128K-token key tensor of the
+    128K prefill workload: one landmark query per chunk, L2 flushed before
+    every call. HBM roofline on K + q' read and k' + b' written."""
+    import torch
+
+    import chunk_sparse_long_landmark_b200 as hils
+    import synth
+    sh = synth.PREFILL_CONFIGS[3]
+    B, Hkv, N, d, S = sh.B, sh.Hkv, sh.N, sh.d, sh.S
+    nC = N // S
+    g = torch.Generator(device=dev).manual_seed(7)
+    K = torch.randn(B, Hkv, N, d, generator=g, device=dev).to(torch.bfloat16)
+    Q = torch.randn(B, Hkv, nC, d, generator=g, device=dev).to(torch.bfloat16)
+    out = (torch.empty(B, Hkv, nC, d, dtype=torch.bfloat16, device=dev),
+           torch.empty(B, Hkv, nC, dtype=torch.float32, device=dev))
+    for _ in range(args.warmup):
+        hils.build_landmarks(K, Q, S, out=out, stream=stream)
+    steps = max(args.steps, 10)
+    evs = [(torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        hils.build_landmarks(K, Q, S, out=out, stream=stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs)) / steps
+    nbytes = 2 * (B * Hkv * N * d + 2 * B * Hkv * nC * d) + 4 * B * Hkv * nC
+    ach = nbytes / (ms * 1e-3) / 1e9
+    del K, Q, out
+    torch.cuda.empty_cache()
+    return {"workload": "landmarks_128k (Prop. 3.1 summaries of the 128K "
+                        "prefill keys, one query per chunk)",
+            "value": ms * 1e3, "unit": "us/call",
+            "roofline": {"bound": "hbm", "achieved": ach,
+                         "peak": peaks["hbm"], "unit": "GB/s",
+                         "frac": ach / peaks["hbm"],
+                         "peak_source": peaks["src"],
+                         "algorithmic_bytes": nbytes},
+            "config": {"B": B, "Hkv": Hkv, "N": N, "d": d, "S": S,
+                       "l2": "flushed before every call"}}
 
 
 def bench_decode(args, dev, stream, flush, world, max_over_ranks, barrier,

@@ -18,7 +18,7 @@ __all__ = [
     "HilsError", "lib", "library_path", "symbols", "status_string",
     "fwd_prefill", "fwd_decode", "prefill_workspace_size",
     "decode_workspace_size", "PrefillArgs", "DecodeArgs", "STATUS",
-    "launch_count", "fwd_decode_noalloc",
+    "launch_count", "fwd_decode_noalloc", "build_landmarks", "LandmarkArgs",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -38,6 +38,7 @@ symbols = [
     "hils_decode_workspace_size", "hils_fwd_prefill", "hils_fwd_decode",
     "hils_prefill_select", "hils_prefill_attend", "hils_decode_select",
     "hils_decode_attend", "hils_launch_count", "hils_fwd_decode_noalloc",
+    "hils_build_landmarks",
 ]
 
 
@@ -67,6 +68,12 @@ class DecodeArgs(ctypes.Structure):
                 ("V", _p), ("Klm", _p), ("bias", _p), ("cache_len", _p),
                 ("O", _p), ("idx", _p), ("sel_score", _p), ("workspace", _p),
                 ("workspace_bytes", ctypes.c_size_t), ("status", _p)]
+
+
+class LandmarkArgs(ctypes.Structure):
+    _fields_ = [("dtype", _i), ("B", _i), ("Hkv", _i), ("N", _i), ("d", _i),
+                ("S", _i), ("Kc", _p), ("Qlm", _p), ("shared_query", _i),
+                ("Klm", _p), ("bias", _p)]
 
 
 _lib = None
@@ -99,6 +106,9 @@ def lib():
             L.hils_fwd_decode_noalloc.restype = ctypes.c_int
             L.hils_fwd_decode_noalloc.argtypes = [ctypes.POINTER(DecodeArgs),
                                                   ctypes.c_void_p]
+            L.hils_build_landmarks.restype = ctypes.c_int
+            L.hils_build_landmarks.argtypes = [ctypes.POINTER(LandmarkArgs),
+                                               ctypes.c_void_p]
             _lib = L
     return _lib
 
@@ -286,3 +296,29 @@ def fwd_decode_noalloc(Q, K, V, Klm, bias, cache_len, head_map, S, W, topk,
     if rc:
         raise HilsError(rc, "hils_fwd_decode_noalloc")
     return out, idx
+
+
+def build_landmarks(K, Qlm, S, out=None, stream=None):
+    """Landmark summaries (k', b') of every full chunk through
+    hils_build_landmarks: K [B,Hkv,N,d]; Qlm [B,Hkv,N//S,d] (one landmark
+    query per chunk) or [Hkv,d] (one shared query per kv head). Returns
+    (Klm [B,Hkv,N//S,d] in K's dtype, bias [B,Hkv,N//S] float32)."""
+    import torch
+    _dev(K, Qlm)
+    B, Hkv, N, d = K.shape
+    nC = N // S
+    shared = 1 if Qlm.dim() == 2 else 0
+    if Qlm.dtype != K.dtype:
+        raise TypeError("Qlm must have K's dtype")
+    if not (K.is_contiguous() and Qlm.is_contiguous()):
+        raise ValueError("K and Qlm must be contiguous")
+    if out is None:
+        out = (torch.empty(B, Hkv, nC, d, dtype=K.dtype, device=K.device),
+               torch.empty(B, Hkv, nC, dtype=torch.float32, device=K.device))
+    Klm, bias = out
+    a = LandmarkArgs(_dtype_code(K), B, Hkv, N, d, S, _ptr(K), _ptr(Qlm),
+                     shared, _ptr(Klm), _ptr(bias))
+    rc = lib().hils_build_landmarks(ctypes.byref(a), _stream_handle(stream))
+    if rc != 0:
+        raise HilsError(rc, "hils_build_landmarks")
+    return Klm, bias

@@ -207,6 +207,42 @@ hils_status hils_decode_attend(const hils_decode_args *args, void *stream);
 hils_status hils_fwd_decode_noalloc(const hils_decode_args *args, void *stream);
 
 /*
+ * Landmark summaries of the chunks: the (k', b') inputs of the scoring step.
+ * "Hierarchical Sparse Attention Done Right", Sec. 3 (answering RQ1, the
+ * surrogate of Eq. 7): for every full chunk c (nC = floor(N/S) of them) of
+ * every (batch, kv head), a landmark query q'_c induces
+ *   p_j  = softmax_j(q'_c . k_j / sqrt(d)),   j = cS .. cS+S-1,
+ *   k'_c = sum_j p_j k_j                      (the weighted key sum),
+ *   b'_c = -sum_j p_j log p_j                 (its entropy, in [0, log S]),
+ * i.e. Attn(q'_c, K_c, K_c). At q = q'_c the surrogate q.k'_c/sqrt(d) + b'_c
+ * equals the exact chunk log-mass. shared_query = 1 is the pages'
+ * landmark-token-free variant (Sec. 4.1): one query per kv head for every
+ * chunk and batch.
+ *
+ * Layout (device pointers, 16-byte aligned, innermost dimension contiguous):
+ *   Kc    [B,Hkv,N,d]              dtype
+ *   Qlm   [B,Hkv,nC,d], or [Hkv,d] when shared_query = 1,   dtype
+ *   Klm   out [B,Hkv,nC,d]         dtype (k' rounded to it)
+ *   bias  out [B,Hkv,nC]           float32
+ * Supported: d in {64, 128}; S in {32, 64, 128, 256}; N >= S.
+ * The caller owns all buffers; nothing is allocated. Asynchronous on
+ * `stream`; argument errors are returned before anything is enqueued
+ * (HILS_ERR_INVALID_ARG, HILS_ERR_UNSUPPORTED, HILS_ERR_MISALIGNED), launch
+ * failures as HILS_ERR_CUDA.
+ */
+typedef struct {
+    int32_t dtype;                  /* hils_dtype of Kc, Qlm, Klm */
+    int32_t B, Hkv, N, d, S;
+    const void *Kc;
+    const void *Qlm;
+    int32_t shared_query;
+    void *Klm;
+    float *bias;
+} hils_landmark_args;
+
+hils_status hils_build_landmarks(const hils_landmark_args *args, void *stream);
+
+/*
  * Number of kernel launches this library has enqueued in this process so far
  * (all devices, all threads). A diagnostic for counting launches per call.
  */

@@ -158,3 +158,26 @@ def test_binding_refuses_cpu_tensors(L):
     with pytest.raises(ValueError):
         hils.fwd_prefill(Q, Q, Q, Q[:, :, :1], torch.zeros(1, 1, 1), [0], 8,
                          8, 1)
+
+
+def _lm_args(**kw):
+    fake = 1 << 40                       # never dereferenced: refused first
+    a = dict(dtype=hils.BF16, B=1, Hkv=2, N=1024, d=128, S=64, Kc=fake,
+             Qlm=fake + 4096, shared_query=0, Klm=fake + 8192,
+             bias=fake + 12288)
+    a.update(kw)
+    return hils.LandmarkArgs(**a)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), 2), (dict(S=48), 2), (dict(S=512), 2),
+    (dict(N=32), 1), (dict(B=0), 1), (dict(dtype=7), 1),
+    (dict(shared_query=2), 1), (dict(Kc=None), 1), (dict(bias=None), 1),
+    (dict(Kc=(1 << 40) + 8), 3), (dict(Klm=(1 << 40) + 4), 3),
+])
+def test_build_landmarks_rejects_before_launch(L, kw, code):
+    assert L.hils_build_landmarks(ctypes.byref(_lm_args(**kw)), None) == code
+
+
+def test_build_landmarks_null_args(L):
+    assert L.hils_build_landmarks(None, None) == 1

@@ -62,42 +62,39 @@ def prefill_work(sh):
 
 
 def union_stats(sh, idx):
-    """Chunk-union diagnostics of the attention tiling (torch on the device).
+    """Chunk-union diagnostics of the attention tiling, counted on the
+    device by the library's hils_chunk_overlap.
 
     The attention kernel gives each block of M = 128/G adjacent queries one
     CTA that loads the union of their selected chunks. Returns the mean union
     size, the pages' chunk-overlap ratio (MK - |union|) / ((M-1)K) (Sec. 7.2)
-    averaged over blocks whose queries all have K selected chunks, and the
+    averaged over blocks whose queries all have K selected chunks, the share
+    of a block's chunks the previous block already had, and the
     executed/touched ratio of the attention MMA work (union + window tiles
     for all 128 rows vs. the algorithmic 4d(|I_i| S + window) per row-head).
     """
     import torch
-    G = sh.G
-    M = 128 // G
+
+    import chunk_sparse_long_landmark_b200 as hils
+    M = 128 // sh.G
     B, Hkv, N, K = idx.shape
-    nqb = (N + M - 1) // M
-    pad = nqb * M - N
-    x = idx
-    if pad:
-        x = torch.cat([x, torch.full((B, Hkv, pad, K), -1, dtype=x.dtype,
-                                     device=x.device)], dim=2)
-    x = x.view(B, Hkv, nqb, M * K)
-    srt, _ = torch.sort(x, dim=-1)
-    new = torch.ones_like(srt, dtype=torch.bool)
-    new[..., 1:] = srt[..., 1:] != srt[..., :-1]
-    union = ((srt >= 0) & new).sum(-1).double()            # [B,Hkv,nqb]
-    full = (x >= 0).sum(-1) == M * K
-    ov = ((M * K - union) / ((M - 1) * K))[full]
+    n_sel, n_union, n_reuse = (t.double() for t in
+                               hils.chunk_overlap(idx, N // sh.S, M))
+    nqb = n_union.shape[-1]
+    full = n_sel == M * K
+    ov = ((M * K - n_union) / ((M - 1) * K))[full]
+    reuse = (n_reuse[..., 1:] / n_union[..., 1:].clamp(min=1)).mean()
     i0 = torch.arange(nqb, device=idx.device, dtype=torch.float64) * M
     il = torch.clamp(i0 + M - 1, max=N - 1)
     w0 = torch.clamp(torch.div(i0 - sh.W + 1, sh.S, rounding_mode="floor") * sh.S, min=0)
     wt = torch.div(il - w0, sh.S, rounding_mode="floor") + 1
     # one CTA = 128 rows (all G heads of M queries) x (union + window) tiles
-    executed = ((union + wt.view(1, 1, -1)) * 128 * sh.S * sh.d * 4).sum().item()
+    executed = ((n_union + wt.view(1, 1, -1)) * 128 * sh.S * sh.d * 4).sum().item()
     touched = prefill_work(sh)["attend_flops"]
-    return {"mean_union_chunks": union.mean().item(),
+    return {"mean_union_chunks": n_union.mean().item(),
             "overlap_M": M,
             "overlap_mean": ov.mean().item() if ov.numel() else None,
+            "reuse_of_previous_block": reuse.item() if nqb > 1 else None,
             "attend_executed_over_touched": executed / touched}
 
 

@@ -19,6 +19,7 @@ __all__ = [
     "fwd_prefill", "fwd_decode", "prefill_workspace_size",
     "decode_workspace_size", "PrefillArgs", "DecodeArgs", "STATUS",
     "launch_count", "fwd_decode_noalloc", "build_landmarks", "LandmarkArgs",
+    "chunk_overlap",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -38,7 +39,7 @@ symbols = [
     "hils_decode_workspace_size", "hils_fwd_prefill", "hils_fwd_decode",
     "hils_prefill_select", "hils_prefill_attend", "hils_decode_select",
     "hils_decode_attend", "hils_launch_count", "hils_fwd_decode_noalloc",
-    "hils_build_landmarks",
+    "hils_build_landmarks", "hils_chunk_overlap",
 ]
 
 
@@ -109,6 +110,8 @@ def lib():
             L.hils_build_landmarks.restype = ctypes.c_int
             L.hils_build_landmarks.argtypes = [ctypes.POINTER(LandmarkArgs),
                                                ctypes.c_void_p]
+            L.hils_chunk_overlap.restype = ctypes.c_int
+            L.hils_chunk_overlap.argtypes = [_p] + [_i] * 6 + [_p] * 4
             _lib = L
     return _lib
 
@@ -322,3 +325,23 @@ def build_landmarks(K, Qlm, S, out=None, stream=None):
     if rc != 0:
         raise HilsError(rc, "hils_build_landmarks")
     return Klm, bias
+
+
+def chunk_overlap(idx, nC, M, stream=None):
+    """Per block of M consecutive query rows of idx [B,Hkv,N,K] (int32, as
+    the select stage writes it): (n_sel, n_union, n_reuse), each
+    [B,Hkv,ceil(N/M)] int32, through hils_chunk_overlap."""
+    import torch
+    _dev(idx)
+    if idx.dtype != torch.int32 or not idx.is_contiguous():
+        raise ValueError("idx must be a contiguous int32 tensor")
+    B, Hkv, N, K = idx.shape
+    nb = (N + M - 1) // M
+    outs = [torch.empty(B, Hkv, nb, dtype=torch.int32, device=idx.device)
+            for _ in range(3)]
+    rc = lib().hils_chunk_overlap(_ptr(idx), B, Hkv, N, K, int(nC), int(M),
+                                  *[_ptr(t) for t in outs],
+                                  _stream_handle(stream))
+    if rc != 0:
+        raise HilsError(rc, "hils_chunk_overlap")
+    return tuple(outs)

@@ -243,6 +243,30 @@ typedef struct {
 hils_status hils_build_landmarks(const hils_landmark_args *args, void *stream);
 
 /*
+ * Chunk-overlap diagnostics of a selection ("Hierarchical Sparse Attention
+ * Done Right", Sec. 7.2: Overlap = (M K - |I_1 u ... u I_M|) / ((M-1) K) for
+ * M adjacent queries). For every block of M consecutive query rows (the last
+ * block may be shorter) of every (batch, kv head):
+ *   n_sel   = entries >= 0 of the block's idx rows,
+ *   n_union = distinct chunks among them,
+ *   n_reuse = distinct chunks also in the previous block's union (0 for the
+ *             first block).
+ * Overlap of a full block whose rows hold K chunks each is
+ * (M*K - n_union) / ((M-1)*K).
+ *   idx      [B,Hkv,N,K] int32, device (as the select stage writes it);
+ *            entries outside [0, nC) other than -1 are an argument error the
+ *            kernel cannot see: they are skipped
+ *   n_sel, n_union, n_reuse   out [B,Hkv,ceil(N/M)] int32, device
+ *   nC       bound on the chunk indices; 2 <= M <= 128; 1 <= K <= 64.
+ * Asynchronous on `stream`; nothing allocated; argument errors returned
+ * before anything is enqueued.
+ */
+hils_status hils_chunk_overlap(const int32_t *idx, int32_t B, int32_t Hkv,
+                               int32_t N, int32_t K, int32_t nC, int32_t M,
+                               int32_t *n_sel, int32_t *n_union,
+                               int32_t *n_reuse, void *stream);
+
+/*
  * Number of kernel launches this library has enqueued in this process so far
  * (all devices, all threads). A diagnostic for counting launches per call.
  */

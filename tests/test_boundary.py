@@ -181,3 +181,21 @@ def test_build_landmarks_rejects_before_launch(L, kw, code):
 
 def test_build_landmarks_null_args(L):
     assert L.hils_build_landmarks(None, None) == 1
+
+
+@pytest.mark.parametrize("args,code", [
+    ((1, 2, 100, 16, 50, 1), 1), ((1, 2, 100, 65, 50, 16), 1),
+    ((1, 2, 100, 16, 0, 16), 1), ((0, 2, 100, 16, 50, 16), 1),
+    ((1, 2, 100, 16, 50, 129), 1),
+])
+def test_chunk_overlap_rejects_before_launch(L, args, code):
+    fake = 1 << 40
+    assert L.hils_chunk_overlap(fake, *args, fake, fake, fake, None) == code
+
+
+def test_chunk_overlap_rejects_null(L):
+    fake = 1 << 40
+    assert L.hils_chunk_overlap(None, 1, 2, 100, 16, 50, 16, fake, fake,
+                                fake, None) == 1
+    assert L.hils_chunk_overlap(fake, 1, 2, 100, 16, 50, 16, fake, None,
+                                fake, None) == 1

@@ -451,7 +451,7 @@ def main():
             "peak_source": peaks["src"],
             "algorithmic_flops_per_launch": dom_flops,
             "traffic": profiled_traffic(
-                ["tc_attend" if dom == "attend" else "tc_score"],
+                ["tc_attend" if dom == "attend" else "tc_select"],
                 args.workload)}
 
     line = {
@@ -567,14 +567,17 @@ def bench_landmarks(args, dev, stream, flush, max_over_ranks, barrier,
     ach = nbytes / (ms * 1e-3) / 1e9
     del K, Q, out
     torch.cuda.empty_cache()
-    return {"workload": "landmarks_128k (Prop. 3.1 summaries of the 128K "
-                        "prefill keys, one query per chunk)",
+    return {"workload": "landmarks_128k",
+            "description": "Prop. 3.1 summaries of the 128K prefill keys, "
+                           "one landmark query per chunk",
             "value": ms * 1e3, "unit": "us/call",
             "roofline": {"bound": "hbm", "achieved": ach,
                          "peak": peaks["hbm"], "unit": "GB/s",
                          "frac": ach / peaks["hbm"],
                          "peak_source": peaks["src"],
-                         "algorithmic_bytes": nbytes},
+                         "algorithmic_bytes": nbytes,
+                         "traffic": profiled_traffic(["landmarks"],
+                                                     "landmarks_128k")},
             "config": {"B": B, "Hkv": Hkv, "N": N, "d": d, "S": S,
                        "l2": "flushed before every call"}}
 

@@ -554,6 +554,7 @@ dec_select_kernel(const DecParams p) {
 // them online per head: running reference max M, O accumulated in the MMA
 // registers (rescaled when M rises), l in registers.
 constexpr int kAttPerMin = 4;                    // tiles per CTA, at least
+constexpr int kAttBuf = 3;                       // K/V tile buffers per CTA
 
 template <int S_TOK, int D>
 __global__ void __launch_bounds__(kAttThreads)
@@ -565,7 +566,7 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     constexpr int NT = TOK_W / 8;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t bar[2];
+    __shared__ uint64_t bar[kAttBuf];
     __shared__ float red[4][8];
     __shared__ float rmx[2][4][8], rsm[2][4][8];
     __shared__ int last;
@@ -598,24 +599,24 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     bool arrived_all = true;
 
     if (threadIdx.x == 0 && nmine > 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
+        for (int k = 0; k < kAttBuf; ++k) mbar_init(&bar[k], 1);
         fence_barrier_init();
     }
     __syncthreads();
-    auto issue = [&](int k) {                    // tile tb + k into buffer k & 1
+    auto issue = [&](int k) {                    // tile tb + k into buffer k % kAttBuf
         const int64_t row = (int64_t)bg * p.Lmax + tile_j0(tb + k);
-        uint8_t *dst = smem + (k & 1) * 2 * TB;
-        mbar_expect_tx(&bar[k & 1], 2 * TB);
+        const int bi = k % kAttBuf;
+        uint8_t *dst = smem + bi * 2 * TB;
+        mbar_expect_tx(&bar[bi], 2 * TB);
         for (int hf = 0; hf < HALVES; ++hf) {
-            tma_load_2d(dst + hf * (S_TOK * 128), &tmK, &bar[k & 1], hf * 64, (int)row);
-            tma_load_2d(dst + TB + hf * (S_TOK * 128), &tmV, &bar[k & 1], hf * 64, (int)row);
+            tma_load_2d(dst + hf * (S_TOK * 128), &tmK, &bar[bi], hf * 64, (int)row);
+            tma_load_2d(dst + TB + hf * (S_TOK * 128), &tmV, &bar[bi], hf * 64, (int)row);
         }
     };
     // window tiles need nothing from the selection: their copies start
     // before the wait for the selection kernel
     if (threadIdx.x == 0)
-        for (int k = 0; k < min(nmine, 2); ++k)
+        for (int k = 0; k < min(nmine, kAttBuf); ++k)
             if (tb + k >= nsel) issue(k);
     grid_dep_wait();                             // dec_select's idx and s^
     // this (b, g)'s selection -- chunk indices and the heads' s^ -- staged
@@ -629,7 +630,7 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     }
     __syncthreads();
     if (threadIdx.x == 0)
-        for (int k = 0; k < min(nmine, 2); ++k)
+        for (int k = 0; k < min(nmine, kAttBuf); ++k)
             if (tb + k < nsel) issue(k);
 
     if (nmine > 0) {
@@ -656,11 +657,11 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
             const int tau = tb + k;
             const bool is_chunk = tau < nsel;
             const int64_t j0 = tile_j0(tau);
-            if (!__syncthreads_and(mbar_wait(&bar[k & 1], (k >> 1) & 1, &dummy_abort) ? 1 : 0)) {
+            if (!__syncthreads_and(mbar_wait(&bar[k % kAttBuf], (k / kAttBuf) & 1, &dummy_abort) ? 1 : 0)) {
                 arrived_all = false;
                 break;
             }
-            const uint32_t sK = smem_u32(smem + (k & 1) * 2 * TB);
+            const uint32_t sK = smem_u32(smem + (k % kAttBuf) * 2 * TB);
             const uint32_t sV = sK + TB;
             float sacc[NT][4];
 #pragma unroll
@@ -762,14 +763,13 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                     mma_bf16(oacc[n + 1], ap, bm[2], bm[3]);
                 }
             }
-            __syncthreads();                     // buffer k & 1 fully read
-            if (threadIdx.x == 0 && k + 2 < nmine) issue(k + 2);
+            __syncthreads();                     // buffer k % kAttBuf fully read
+            if (threadIdx.x == 0 && k + kAttBuf < nmine) issue(k + kAttBuf);
         }
         if (!arrived_all) {
             if (threadIdx.x == 0) {
                 report(p.status, HILS_ERR_DEVICE_TIMEOUT);
-                mbar_drain(&bar[0], 0);
-                mbar_drain(&bar[1], 0);
+                for (int k = 0; k < kAttBuf; ++k) mbar_drain(&bar[k], 0);
             }
             __syncthreads();
             return;                              // no ticket: O stays unwritten
@@ -812,22 +812,26 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     if (!last || !ok) return;
     __threadfence();
     const int ngrp = (ntot + p.att_per - 1) / p.att_per;
-    // per group and head: w_gg / sum_gg' w_gg' l_gg' with w = exp(m - max m)
-    // (the stage buffers are free now), then O = sum of weighted partial O
-    // in group order, the partial loads of 8 groups issued together
-    float *cw = reinterpret_cast<float *>(smem);             // [ngrp][G]
+    // per group and head: w_gg / sum_gg' w_gg' l_gg' with w = exp(m - max m).
+    // All (m, l) partials of this (b, g) come in with one round trip (the
+    // stage buffers are free now), then O = sum of weighted partial O in
+    // group order, the partial loads of 8 groups issued together.
+    float *cml = reinterpret_cast<float *>(smem);            // [ngrp][G][2]
+    float *cw = cml + 2 * ngrp * G;                          // [ngrp][G]
+    {
+        const float *src = p.ws_ml + (int64_t)bg * p.ntile * G * 2;
+        for (int e = threadIdx.x; e < 2 * ngrp * G; e += kAttThreads) cml[e] = __ldcg(src + e);
+    }
+    __syncthreads();
     if (threadIdx.x < G) {
         const int hh = threadIdx.x;
-        const float *mlb = p.ws_ml + ((int64_t)bg * p.ntile * G + hh) * 2;
         float M = -INFINITY;
-#pragma unroll 8
-        for (int gg = 0; gg < ngrp; ++gg) M = fmaxf(M, __ldcg(mlb + (int64_t)gg * G * 2));
+        for (int gg = 0; gg < ngrp; ++gg) M = fmaxf(M, cml[(gg * G + hh) * 2]);
         float den = 0.f;
-#pragma unroll 8
         for (int gg = 0; gg < ngrp; ++gg) {
-            const float w = exp2f((__ldcg(mlb + (int64_t)gg * G * 2) - M) * kLog2e);
+            const float w = exp2f((cml[(gg * G + hh) * 2] - M) * kLog2e);
             cw[gg * G + hh] = w;
-            den += w * __ldcg(mlb + (int64_t)gg * G * 2 + 1);
+            den += w * cml[(gg * G + hh) * 2 + 1];
         }
         const float inv = 1.f / den;
         for (int gg = 0; gg < ngrp; ++gg) cw[gg * G + hh] *= inv;
@@ -1007,8 +1011,8 @@ cudaError_t launch_dec_select(Problem &p, void *ws, cudaStream_t st) {
 template <int S_TOK, int D>
 cudaError_t launch_att_t(const DecParams &d, const CUtensorMap &tk,
                          const CUtensorMap &tv, cudaStream_t st) {
-    static_assert(4 * 8 * D * 4 <= 4 * S_TOK * D * 2, "partial O fits the stages");
-    const size_t smem = 1024 + 4ull * S_TOK * D * 2;
+    static_assert(4 * 8 * D * 4 <= 2 * kAttBuf * S_TOK * D * 2, "partial O fits the stages");
+    const size_t smem = 1024 + 2ull * kAttBuf * S_TOK * D * 2;
     cudaError_t e = cudaFuncSetAttribute(dec_attend_kernel<S_TOK, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);

@@ -19,7 +19,7 @@ __all__ = [
     "fwd_prefill", "fwd_decode", "prefill_workspace_size",
     "decode_workspace_size", "PrefillArgs", "DecodeArgs", "STATUS",
     "launch_count", "fwd_decode_noalloc", "build_landmarks", "LandmarkArgs",
-    "chunk_overlap",
+    "chunk_overlap", "fwd_decode_paged", "DecodePagedArgs",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -40,6 +40,7 @@ symbols = [
     "hils_prefill_select", "hils_prefill_attend", "hils_decode_select",
     "hils_decode_attend", "hils_launch_count", "hils_fwd_decode_noalloc",
     "hils_build_landmarks", "hils_chunk_overlap",
+    "hils_decode_paged_workspace_size", "hils_fwd_decode_paged",
 ]
 
 
@@ -69,6 +70,10 @@ class DecodeArgs(ctypes.Structure):
                 ("V", _p), ("Klm", _p), ("bias", _p), ("cache_len", _p),
                 ("O", _p), ("idx", _p), ("sel_score", _p), ("workspace", _p),
                 ("workspace_bytes", ctypes.c_size_t), ("status", _p)]
+
+
+class DecodePagedArgs(ctypes.Structure):
+    _fields_ = [("base", DecodeArgs), ("block_table", _p), ("n_pages", _i)]
 
 
 class LandmarkArgs(ctypes.Structure):
@@ -110,6 +115,12 @@ def lib():
             L.hils_build_landmarks.restype = ctypes.c_int
             L.hils_build_landmarks.argtypes = [ctypes.POINTER(LandmarkArgs),
                                                ctypes.c_void_p]
+            L.hils_decode_paged_workspace_size.restype = ctypes.c_int
+            L.hils_decode_paged_workspace_size.argtypes = [
+                ctypes.POINTER(DecodePagedArgs), ctypes.POINTER(ctypes.c_size_t)]
+            L.hils_fwd_decode_paged.restype = ctypes.c_int
+            L.hils_fwd_decode_paged.argtypes = [ctypes.POINTER(DecodePagedArgs),
+                                                ctypes.c_void_p]
             L.hils_chunk_overlap.restype = ctypes.c_int
             L.hils_chunk_overlap.argtypes = [_p] + [_i] * 6 + [_p] * 4
             _lib = L
@@ -345,3 +356,52 @@ def chunk_overlap(idx, nC, M, stream=None):
     if rc != 0:
         raise HilsError(rc, "hils_chunk_overlap")
     return tuple(outs)
+
+
+def fwd_decode_paged(Q, Kpool, Vpool, Klm, bias, cache_len, block_table,
+                     head_map, S, W, topk, Qs=None, out=None, idx=None,
+                     sel_score=None, workspace=None, status=None,
+                     stream=None):
+    """HiLS decode step over a paged cache (page = chunk) through
+    hils_fwd_decode_paged. Returns (O, idx).
+
+    Kpool/Vpool [n_pages,Hkv,S,d]; block_table int32 [B, Lmax//S] on the
+    device (page of each logical chunk); Klm [B,Hkv,Lmax//S,d] and bias
+    [B,Hkv,Lmax//S] per sequence; cache_len int32 [B] on the device."""
+    import torch
+    _dev(Q, Kpool, Vpool, Klm, bias, cache_len, block_table, Qs, out, idx,
+         sel_score, workspace, status)
+    if block_table.dtype != torch.int32 or not block_table.is_contiguous():
+        raise ValueError("block_table must be a contiguous int32 tensor")
+    B, Hq, d = Q.shape
+    P, Hkv = Kpool.shape[0], Kpool.shape[1]
+    Lmax = block_table.shape[1] * S
+    hm = _head_map_array(head_map, Hq)
+    if out is None:
+        out = torch.empty_like(Q)
+    if idx is None:
+        idx = torch.empty(B, Hkv, topk, dtype=torch.int32, device=Q.device)
+
+    def record(ws):
+        base = DecodeArgs(_dtype_code(Q), B, Hq, Hkv, Lmax, d, S, W, topk,
+                          ctypes.cast(hm, ctypes.c_void_p), _ptr(Q), _ptr(Qs),
+                          _ptr(Kpool), _ptr(Vpool), _ptr(Klm), _ptr(bias),
+                          _ptr(cache_len), _ptr(out), _ptr(idx),
+                          _ptr(sel_score), _ptr(ws),
+                          0 if ws is None else ws.numel() * ws.element_size(),
+                          _ptr(status))
+        return DecodePagedArgs(base, _ptr(block_table), P)
+
+    if workspace is None:
+        n = ctypes.c_size_t(0)
+        rc = lib().hils_decode_paged_workspace_size(ctypes.byref(record(None)),
+                                                    ctypes.byref(n))
+        if rc:
+            raise HilsError(rc, "hils_decode_paged_workspace_size")
+        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8,
+                                device=Q.device)
+    a = record(workspace)
+    rc = lib().hils_fwd_decode_paged(ctypes.byref(a), _stream_handle(stream))
+    if rc:
+        raise HilsError(rc, "hils_fwd_decode_paged")
+    return out, idx

@@ -43,6 +43,8 @@ struct DecParams {
     const void *Q, *Qs;
     const float *bias;
     const int32_t *cache_len;
+    const int32_t *block_table;  // paged cache: [B, Lmax/S] page of each chunk
+    int n_pages;
     void *O;
     int32_t *idx;
     float *sel;
@@ -603,8 +605,20 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
         fence_barrier_init();
     }
     __syncthreads();
+    // TMA row of a tile: contiguous cache [B,Hkv,Lmax,d], or the page pool
+    // [n_pages,Hkv,S,d] (a tile is one chunk, i.e. one page)
+    auto tile_row = [&](int tau) -> int64_t {
+        const int64_t j0 = tile_j0(tau);
+        if (!p.block_table) return (int64_t)bg * p.Lmax + j0;
+        const int pg = p.block_table[(int64_t)b * (p.Lmax / p.S) + j0 / p.S];
+        if (pg < 0 || pg >= p.n_pages) {         // a box wholly before row 0:
+            report(p.status, HILS_ERR_DEVICE_BAD_LENGTH);   // TMA reads zeros
+            return -(int64_t)p.S;
+        }
+        return ((int64_t)pg * p.Hkv + g) * p.S;
+    };
     auto issue = [&](int k) {                    // tile tb + k into buffer k % kAttBuf
-        const int64_t row = (int64_t)bg * p.Lmax + tile_j0(tb + k);
+        const int64_t row = tile_row(tb + k);
         const int bi = k % kAttBuf;
         uint8_t *dst = smem + bi * 2 * TB;
         mbar_expect_tx(&bar[bi], 2 * TB);
@@ -932,6 +946,7 @@ DecParams dec_params(const Problem &p, void *ws) {
     DecParams d;
     char *base = (char *)ws;
     d.Q = p.Q; d.Qs = p.Qs; d.bias = p.bias; d.cache_len = p.cache_len;
+    d.block_table = p.block_table; d.n_pages = p.n_pages;
     d.O = p.O; d.idx = p.idx; d.sel = p.sel; d.status = p.status;
     d.ws_s = (float *)(base + pl.off_s);
     d.ws_p = (float *)(base + pl.off_p);
@@ -1026,7 +1041,8 @@ cudaError_t launch_att_t(const DecParams &d, const CUtensorMap &tk,
 cudaError_t launch_dec_attend(Problem &p, void *ws, cudaStream_t st) {
     DecParams d = dec_params(p, ws);
     CUtensorMap tk, tv;
-    const int64_t rows = (int64_t)p.B * p.Hkv * p.kv_rows;
+    const int64_t rows = p.block_table ? (int64_t)p.n_pages * p.Hkv * p.S
+                                       : (int64_t)p.B * p.Hkv * p.kv_rows;
     if (!map_2d(&tk, p.Kc, p.d, rows, p.S) || !map_2d(&tv, p.V, p.d, rows, p.S))
         return cudaErrorInvalidValue;
     cudaError_t e;

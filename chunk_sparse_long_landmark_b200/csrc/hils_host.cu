@@ -193,6 +193,24 @@ hils_status prefill_entry(const hils_prefill_args *args, void *stream,
                (cudaStream_t)stream, stages);
 }
 
+// The paged record: the decode record's checks, plus the page table, and
+// only the shapes the HBM decode kernels run.
+hils_status paged_problem(const hils_decode_paged_args *a, Problem *p,
+                          bool need_ptrs) {
+    if (!a) return HILS_ERR_INVALID_ARG;
+    hils_status s = decode_problem(&a->base, p, need_ptrs);
+    if (s != HILS_OK) return s;
+    if (a->base.Lmax % a->base.S != 0 || a->n_pages < 1) return HILS_ERR_INVALID_ARG;
+    if ((int64_t)a->n_pages * a->base.Hkv * a->base.S >= (1ll << 31))
+        return HILS_ERR_UNSUPPORTED;                 // TMA row coordinates are int32
+    if (need_ptrs && !a->block_table) return HILS_ERR_INVALID_ARG;
+    p->block_table = a->block_table;
+    p->n_pages = a->n_pages;
+    if (!fast_path_supported(*p) || !fast_select_supported(*p))
+        return HILS_ERR_UNSUPPORTED;
+    return HILS_OK;
+}
+
 hils_status decode_entry(const hils_decode_args *args, void *stream,
                          int stages) {
     Problem p;
@@ -278,6 +296,28 @@ hils_status hils_decode_select(const hils_decode_args *args, void *stream) {
 
 hils_status hils_decode_attend(const hils_decode_args *args, void *stream) {
     return decode_entry(args, stream, kAttend);
+}
+
+hils_status hils_decode_paged_workspace_size(const hils_decode_paged_args *args,
+                                             size_t *bytes) {
+    if (!bytes) return HILS_ERR_INVALID_ARG;
+    Problem p;
+    hils_status s = paged_problem(args, &p, false);
+    if (s != HILS_OK) return s;
+    Plan pl;
+    plan_workspace(p, args->base.sel_score != nullptr, &pl);
+    *bytes = pl.total;
+    return HILS_OK;
+}
+
+hils_status hils_fwd_decode_paged(const hils_decode_paged_args *args, void *stream) {
+    Problem p;
+    hils_status s = paged_problem(args, &p, true);
+    if (s != HILS_OK) return s;
+    Plan pl;
+    plan_workspace(p, args->base.sel_score != nullptr, &pl);
+    return run(p, pl, args->base.workspace, args->base.workspace_bytes,
+               (cudaStream_t)stream, kBoth);
 }
 
 uint64_t hils_launch_count(void) { return launch_total(); }

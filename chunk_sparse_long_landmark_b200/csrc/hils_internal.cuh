@@ -22,6 +22,8 @@ struct Problem {
     int32_t *idx;
     float *sel;                  // s^ of the selected chunks [B,Hq,n_query,K]
     const int32_t *cache_len;    // decode only
+    const int32_t *block_table;  // decode over a paged cache: [B, kv_rows/S]
+    int n_pages;                 // pages of S tokens in the pool (paged only)
     int32_t *status;             // nullable
     int B, Hq, Hkv, G, d, S, W, K;
     int n_query;                 // query rows per (b, h): N or 1

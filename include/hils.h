@@ -207,6 +207,35 @@ hils_status hils_decode_attend(const hils_decode_args *args, void *stream);
 hils_status hils_fwd_decode_noalloc(const hils_decode_args *args, void *stream);
 
 /*
+ * Decode over a paged KV cache with page = chunk ("Hierarchical Sparse
+ * Attention Done Right", Sec. 7.1: the serving setup keeps the cache in
+ * pages of one chunk). Same computation and outputs as hils_fwd_decode;
+ * only where K and V live changes:
+ *   base.Kc, base.V   the page pool [n_pages, Hkv, S, d] (dtype): page p
+ *                     holds S consecutive tokens of every kv head
+ *   block_table       device int32 [B, base.Lmax / S]: the page holding
+ *                     logical chunk c (tokens cS .. cS+S-1) of sequence b;
+ *                     only the chunks a step reads (the selected ones and
+ *                     the window's) need valid entries
+ *   n_pages           pages in the pool
+ * base.Lmax is the logical capacity per sequence (a multiple of S); the
+ * landmark tensors Klm [B,Hkv,Lmax/S,d] and bias stay per sequence, as in
+ * hils_fwd_decode. Supported: bf16, d in {64,128}, S in {64,128}, G <= 8
+ * (the HBM decode kernels); other shapes return HILS_ERR_UNSUPPORTED. A page
+ * index outside [0, n_pages) reads zeros and raises
+ * HILS_ERR_DEVICE_BAD_LENGTH in the status word.
+ */
+typedef struct {
+    hils_decode_args base;
+    const int32_t *block_table;
+    int32_t n_pages;
+} hils_decode_paged_args;
+
+hils_status hils_decode_paged_workspace_size(const hils_decode_paged_args *args,
+                                             size_t *bytes);
+hils_status hils_fwd_decode_paged(const hils_decode_paged_args *args, void *stream);
+
+/*
  * Landmark summaries of the chunks: the (k', b') inputs of the scoring step.
  * "Hierarchical Sparse Attention Done Right", Sec. 3 (answering RQ1, the
  * surrogate of Eq. 7): for every full chunk c (nC = floor(N/S) of them) of

@@ -199,3 +199,38 @@ def test_chunk_overlap_rejects_null(L):
                                 fake, None) == 1
     assert L.hils_chunk_overlap(fake, 1, 2, 100, 16, 50, 16, fake, None,
                                 fake, None) == 1
+
+
+def _paged(**kw):
+    fake = 1 << 40
+    base = hils.DecodeArgs(hils.BF16, 2, 8, 2, 1024, 128, 64, 128, 8,
+                           None, fake, None, fake, fake, fake, fake, fake,
+                           fake, fake, None, fake, 1 << 30, None)
+    a = dict(base=base, block_table=fake, n_pages=40)
+    a.update(kw)
+    return hils.DecodePagedArgs(**a)
+
+
+def test_decode_paged_validation(L):
+    hm = (ctypes.c_int32 * 8)(*[h // 4 for h in range(8)])
+    a = _paged()
+    a.base.head_map = ctypes.cast(hm, ctypes.c_void_p)
+    n = ctypes.c_size_t(0)
+    # without a CUDA driver (CPU-only host) the HBM kernels report
+    # themselves unavailable: HILS_ERR_UNSUPPORTED; with one, a size
+    rc = L.hils_decode_paged_workspace_size(ctypes.byref(a), ctypes.byref(n))
+    assert rc in (0, 2)
+    assert rc == 2 or n.value > 0
+    for kw, code in [(dict(block_table=None), 1), (dict(n_pages=0), 1)]:
+        b = _paged(**kw)
+        b.base.head_map = ctypes.cast(hm, ctypes.c_void_p)
+        assert L.hils_fwd_decode_paged(ctypes.byref(b), None) == code
+    c = _paged()
+    c.base.head_map = ctypes.cast(hm, ctypes.c_void_p)
+    c.base.Lmax = 1000                    # not a multiple of S
+    assert L.hils_fwd_decode_paged(ctypes.byref(c), None) == 1
+    d = _paged()
+    d.base.head_map = ctypes.cast(hm, ctypes.c_void_p)
+    d.base.dtype = hils.F32               # no f32 paged kernels
+    assert L.hils_fwd_decode_paged(ctypes.byref(d), None) == 2
+    assert L.hils_fwd_decode_paged(None, None) == 1

@@ -130,3 +130,54 @@ def test_decode_exact_score_ties_take_lower_chunks(every, cuda_device):
         for g in range(sh.Hkv):
             np.testing.assert_array_equal(got[b, g], want)
     parity.check_decode(inp, O, idx)
+
+
+def _to_pages(inp, sh, seed, spare=5):
+    """Scatter the contiguous caches into a shuffled page pool (page = one
+    chunk of every kv head) with a random block table, plus unused pages."""
+    B, Hkv, L, d = inp["K"].shape
+    npg = L // sh.S
+    P = B * npg + spare
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    perm = torch.randperm(P, generator=g)[:B * npg].view(B, npg)
+    dev = inp["K"].device
+    bt = perm.to(torch.int32).to(dev).contiguous()
+    pools = []
+    for name in ("K", "V"):
+        pool = torch.randn(P, Hkv, sh.S, d, device=dev).to(inp[name].dtype)
+        x = inp[name].view(B, Hkv, npg, sh.S, d).permute(0, 2, 1, 3, 4)
+        pool[perm.reshape(-1).to(dev)] = x.reshape(B * npg, Hkv, sh.S, d)
+        pools.append(pool.contiguous())
+    return pools[0], pools[1], bt
+
+
+@pytest.mark.parametrize("name", ["bf16_ragged", "bf16_d64_S128", "bf16_short"])
+def test_decode_paged_equals_contiguous(name, cuda_device):
+    """Same kernels, addressed through a block table: the paged step gives
+    bit-identical O and idx to the contiguous one, and matches the oracle."""
+    sh, lens = CASES[name]
+    inp = synth.make_decode(sh, seed=205, device=cuda_device, cache_len=lens)
+    O_ref, idx_ref = run_decode(inp)
+    Kp, Vp, bt = _to_pages(inp, sh, seed=7)
+    O, idx = hils.fwd_decode_paged(inp["Q"], Kp, Vp, inp["Klm"], inp["bias"],
+                                   inp["cache_len"], bt, inp["head_map"],
+                                   sh.S, sh.W, sh.K)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx_ref)
+    assert torch.equal(O, O_ref)
+    parity.check_decode(inp, O, idx)
+
+
+def test_decode_paged_bad_page_reported(cuda_device):
+    """A page index outside the pool is reported in the status word (and
+    read as zeros): no fault."""
+    sh, lens = CASES["bf16_short"]
+    inp = synth.make_decode(sh, seed=206, device=cuda_device, cache_len=lens)
+    Kp, Vp, bt = _to_pages(inp, sh, seed=8)
+    bt[0, (lens[0] - 1) // sh.S] = Kp.shape[0] + 3      # the query's own page
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    hils.fwd_decode_paged(inp["Q"], Kp, Vp, inp["Klm"], inp["bias"],
+                          inp["cache_len"], bt, inp["head_map"], sh.S, sh.W,
+                          sh.K, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 7          # HILS_ERR_DEVICE_BAD_LENGTH

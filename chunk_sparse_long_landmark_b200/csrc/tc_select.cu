@@ -348,6 +348,7 @@ tc_select_kernel(const __grid_constant__ CUtensorMap tmL,
         epi_bar();                  // staging is read before the lists overwrite it
 
         const float sl2 = p.inv_sqrt_d * kLog2e;
+        const float2 sl2v = make_float2(sl2, sl2);
         float *bias_w = bias_s + quad * (2 * kTc);
         const float *bias_g = p.bias + ((int64_t)b * p.Hkv + g) * p.nC;
         float bnext = 0.f;
@@ -398,12 +399,21 @@ tc_select_kernel(const __grid_constant__ CUtensorMap tmL,
                     tc_fence_before();
                     mbar_arrive(&st.s_empty[t & 1]);
                 }
+                // x = S/sqrt(d) + b' for column pairs (f32x2: each element
+                // rounded as the scalar fma, so pass 2 forms the same x)
                 float x[G][16];
 #pragma unroll
-                for (int hh = 0; hh < G; ++hh)
+                for (int k = 0; k < 8; ++k) {
+                    const float2 b2 = *reinterpret_cast<const float2 *>(bw + j0 + 2 * k);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        x[hh][j] = fmaf(__uint_as_float(raw[hh][j]), sl2, bw[j0 + j]);
+                    for (int hh = 0; hh < G; ++hh) {
+                        const float2 v = f2_fma(make_float2(__uint_as_float(raw[hh][2 * k]),
+                                                            __uint_as_float(raw[hh][2 * k + 1])),
+                                                sl2v, b2);
+                        x[hh][2 * k] = v.x;
+                        x[hh][2 * k + 1] = v.y;
+                    }
+                }
                 if (edge) {
 #pragma unroll
                     for (int hh = 0; hh < G; ++hh)
@@ -421,11 +431,17 @@ tc_select_kernel(const __grid_constant__ CUtensorMap tmL,
                     for (int j = 0; j < 4; ++j) t8[j] = fmaxf(t8[j], t8[j + 4]);
                     const float mt = fmaxf(fmaxf(t8[0], t8[2]), fmaxf(t8[1], t8[3]));
                     const float mn = fmaxf(mrun[hh], mt);
-                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                    const float2 nm2 = make_float2(-mn, -mn);
+                    float2 acc[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) acc[j & 3] += fast_exp2(x[hh][j] - mn);
+                    for (int k = 0; k < 8; ++k) {
+                        float2 e = f2_add(make_float2(x[hh][2 * k], x[hh][2 * k + 1]), nm2);
+                        e.x = fast_exp2(e.x);
+                        e.y = fast_exp2(e.y);
+                        acc[k & 1] = f2_add(acc[k & 1], e);
+                    }
                     srun[hh] = fmaf(srun[hh], fast_exp2(mrun[hh] - mn),
-                                    (acc[0] + acc[1]) + (acc[2] + acc[3]));
+                                    (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y));
                     mrun[hh] = mn;
                 }
 #pragma unroll
@@ -458,6 +474,9 @@ tc_select_kernel(const __grid_constant__ CUtensorMap tmL,
         }
 
         // ---------------------------------------------------------- pass 2
+        float2 nl2[G];                          // -L_h, twice
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) nl2[hh] = make_float2(-lse2[hh], -lse2[hh]);
         int cnt = 0;
         for (int t = nT; ok && t < T; ++t) {
             const float *bw = stage_bias(t);
@@ -486,22 +505,36 @@ tc_select_kernel(const __grid_constant__ CUtensorMap tmL,
                     tau = nextafterf(mn, INFINITY);
                 }
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    float x[G];
+                for (int k = 0; k < 8; ++k) {
+                    // x and a = max_h (x_h - L_h) for the column pair 2k, 2k+1
+                    const float2 b2 = *reinterpret_cast<const float2 *>(bw + j0 + 2 * k);
+                    float2 x2[G];
 #pragma unroll
                     for (int hh = 0; hh < G; ++hh)
-                        x[hh] = fmaf(__uint_as_float(raw[hh][j]), sl2, bw[j0 + j]);
-                    float a = x[0] - lse2[0];
+                        x2[hh] = f2_fma(make_float2(__uint_as_float(raw[hh][2 * k]),
+                                                    __uint_as_float(raw[hh][2 * k + 1])),
+                                        sl2v, b2);
+                    float2 a2 = f2_add(x2[0], nl2[0]);
 #pragma unroll
-                    for (int hh = 1; hh < G; ++hh) a = fmaxf(a, x[hh] - lse2[hh]);
-                    const bool take = (j0 + j < lim) && (a >= tau);
-                    if (take) {
-                        ca[cnt * kLd + r] = a;
-                        cc[cnt * kLd + r] = c0 + j0 + j;
-#pragma unroll
-                        for (int hh = 0; hh < G; ++hh) cx[(hh * CAP + cnt) * kLd + r] = x[hh];
+                    for (int hh = 1; hh < G; ++hh) {
+                        const float2 v = f2_add(x2[hh], nl2[hh]);
+                        a2.x = fmaxf(a2.x, v.x);
+                        a2.y = fmaxf(a2.y, v.y);
                     }
-                    cnt += take ? 1 : 0;
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int j = 2 * k + e;
+                        const float a = e ? a2.y : a2.x;
+                        const bool take = (j0 + j < lim) && (a >= tau);
+                        if (take) {
+                            ca[cnt * kLd + r] = a;
+                            cc[cnt * kLd + r] = c0 + j0 + j;
+#pragma unroll
+                            for (int hh = 0; hh < G; ++hh)
+                                cx[(hh * CAP + cnt) * kLd + r] = e ? x2[hh].y : x2[hh].x;
+                        }
+                        cnt += take ? 1 : 0;
+                    }
                 }
             }
         }

@@ -16,7 +16,10 @@
 //                    the S columns
 //   O  += P V        tcgen05.mma, 128 x d, A = P from TMEM, f32 in TMEM
 // Shared memory holds only Q and a 2-stage K/V ring (~105 KB) and TMEM 256
-// columns, so two CTAs share an SM and hide each other's latencies.
+// columns, so two CTAs share an SM and hide each other's latencies. A K
+// stage is handed back when its QK product completes and a V stage when its
+// PV product does, so the copy of K runs ahead and two copies of V are in
+// flight behind the PV chain.
 // Warp roles: warp 0 TMA producer (K, V), warp 1 MMA issuer (and TMEM
 // owner), warps 2-5 Q loader, softmax and epilogue (warp w reads TMEM lanes
 // 32*(w%4)..+31). Elementwise softmax arithmetic uses packed f32x2 ops.
@@ -56,8 +59,10 @@ struct AttnLayout {
 
 struct SmallState {
     uint64_t q_full;
-    uint64_t kv_full[kStages];
-    uint64_t kv_empty[kStages];
+    uint64_t k_full[kStages];
+    uint64_t v_full[kStages];
+    uint64_t k_empty[kStages];                       // QK of that stage done
+    uint64_t v_empty[kStages];                       // PV of that stage done
     uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t p_empty[2];                             // PV of that buffer done
@@ -96,8 +101,10 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     if (threadIdx.x == 0) {
         mbar_init(&st.q_full, 128);             // the softmax threads load Q
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&st.kv_full[s], 1);
-            mbar_init(&st.kv_empty[s], 1);
+            mbar_init(&st.k_full[s], 1);
+            mbar_init(&st.v_full[s], 1);
+            mbar_init(&st.k_empty[s], 1);
+            mbar_init(&st.v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&st.s_full[s], 1);
@@ -192,30 +199,47 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     } else if (warp == 0) {
         // ------------------------------------------------------ producer
         if (lane == 0) {
-            int issued = 0;
-            for (int t = 0; t < T; ++t) {
+            // K of a stage is free once the QK product of its tile is done,
+            // V once the PV product is: K copies run ahead of V copies, and
+            // two V copies stay in flight behind the PV chain.
+            auto load = [&](int t, bool is_v) {
                 const int s = t % kStages;
-                if (t >= kStages &&
-                    !mbar_wait(&st.kv_empty[s], ((t / kStages) - 1) & 1, abort))
-                    break;
                 const int row = (t < U) ? s_union[t] * p.S
                                         : wstart + (t - U) * S_TOK;
-                mbar_expect_tx(&st.kv_full[s], 2 * L::KV_BYTES);
-                for (int dh = 0; dh < D / 64; ++dh) {
-                    tma_load_4d(smem + L::OFF_K + s * L::KV_BYTES +
+                uint64_t *bar = is_v ? &st.v_full[s] : &st.k_full[s];
+                mbar_expect_tx(bar, L::KV_BYTES);
+                for (int dh = 0; dh < D / 64; ++dh)
+                    tma_load_4d(smem + (is_v ? L::OFF_V : L::OFF_K) + s * L::KV_BYTES +
                                     dh * (S_TOK * 128),
-                                &tmK, &st.kv_full[s], dh * 64, row, g, b);
-                    tma_load_4d(smem + L::OFF_V + s * L::KV_BYTES +
-                                    dh * (S_TOK * 128),
-                                &tmV, &st.kv_full[s], dh * 64, row, g, b);
+                                is_v ? &tmV : &tmK, bar, dh * 64, row, g, b);
+            };
+            int nk = 0, nv = 0;                          // copies issued
+            while (nv < T) {
+                // next K copy whose stage is already free, else the next V copy
+                if (nk < T && nk < nv + kStages &&
+                    (nk < kStages ||
+                     mbar_try(smem_u32(&st.k_empty[nk % kStages]), ((nk / kStages) - 1) & 1))) {
+                    load(nk++, false);
+                    continue;
                 }
-                issued = t + 1;
+                if (nv < nk) {
+                    if (nv >= kStages &&
+                        !mbar_wait(&st.v_empty[nv % kStages], ((nv / kStages) - 1) & 1, abort))
+                        break;
+                    load(nv++, true);
+                    continue;
+                }
+                // nv == nk: the K copy must go first
+                if (!mbar_wait(&st.k_empty[nk % kStages], ((nk / kStages) - 1) & 1, abort))
+                    break;
+                load(nk++, false);
             }
             // on abort: let the copies already issued land before exiting
             if (*abort) {
-                for (int t = (issued > kStages ? issued - kStages : 0);
-                     t < issued; ++t)
-                    mbar_drain(&st.kv_full[t % kStages], (t / kStages) & 1);
+                for (int t = (nk > kStages ? nk - kStages : 0); t < nk; ++t)
+                    mbar_drain(&st.k_full[t % kStages], (t / kStages) & 1);
+                for (int t = (nv > kStages ? nv - kStages : 0); t < nv; ++t)
+                    mbar_drain(&st.v_full[t % kStages], (t / kStages) & 1);
             }
         }
     } else if (warp == 1) {
@@ -231,8 +255,9 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
             auto do_pv = [&](int u) -> bool {
                 const int pb = u & 1;
                 if (!mbar_wait(&st.p_full[pb], (u >> 1) & 1, abort)) return false;
-                tc_fence_after();
                 const int s = u % kStages;
+                if (!mbar_wait(&st.v_full[s], (u / kStages) & 1, abort)) return false;
+                tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < S_TOK / 16; ++k) {
                     // A = P of this tile, bf16 in the S buffer: 8 columns per 16 tokens
@@ -241,14 +266,14 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                         sV + s * L::KV_BYTES + k * 16 * 128, S_TOK * 128, 1024);
                     mma_ts(tmem + L::TMEM_O, at, bd, id_o, (u > 0 || k > 0) ? 1u : 0u);
                 }
-                mma_commit(&st.kv_empty[s]);
+                mma_commit(&st.v_empty[s]);
                 mma_commit(&st.p_empty[pb]);
                 return true;
             };
             for (int t = 0; ok && t < T; ++t) {
                 const int s = t % kStages;
                 const int sb = t & 1;
-                if (!mbar_wait(&st.kv_full[s], (t / kStages) & 1, abort)) { ok = false; break; }
+                if (!mbar_wait(&st.k_full[s], (t / kStages) & 1, abort)) { ok = false; break; }
                 // S buffer sb is free once PV(t-2), which read its P, is done
                 if (t >= 2 && !mbar_wait(&st.p_empty[sb], ((t - 2) >> 1) & 1, abort)) { ok = false; break; }
                 tc_fence_after();
@@ -262,6 +287,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                     mma_ss(tmem + L::TMEM_S + sb * S_TOK, ad, bd, id_s, k > 0 ? 1u : 0u);
                 }
                 mma_commit(&st.s_full[sb]);
+                mma_commit(&st.k_empty[s]);
                 if (t >= 1 && !do_pv(t - 1)) { ok = false; break; }
             }
             if (ok && T > 0) do_pv(T - 1);

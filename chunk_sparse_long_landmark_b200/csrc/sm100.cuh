@@ -55,6 +55,17 @@ __device__ __forceinline__ bool mbar_try(uint32_t addr, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking probe: has the phase with `parity` completed?
+__device__ __forceinline__ bool mbar_test(uint32_t addr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(addr), "r"(parity) : "memory");
+    return ok != 0;
+}
+
 // Time limit of one wait: far above any legitimate intra-CTA wait.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 

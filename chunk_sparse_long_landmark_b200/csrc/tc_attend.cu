@@ -42,6 +42,26 @@ constexpr int kStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;      // lazy O rescale threshold (log2)
 
+// max over n >= 8 scores (n a multiple of 4), four independent chains
+__device__ __forceinline__ float row_max(const uint32_t *rr, int n) {
+    float m[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m[k] = __uint_as_float(rr[k]);
+#pragma unroll
+    for (int j = 4; j < n; j += 4)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) m[k] = fmaxf(m[k], __uint_as_float(rr[j + k]));
+    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+// a += the two bf16 halves of a packed pair (mixed-precision adds: no
+// unpacking instructions; each sum rounds as the f32 add of the widened value)
+__device__ __forceinline__ void acc_bf16x2(float2 &a, uint32_t v) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(a.x), "+f"(a.y) : "r"(v));
+}
+
 template <int S_TOK, int D>
 struct AttnLayout {
     static constexpr uint32_t Q_BYTES = kRows * D * 2;
@@ -218,7 +238,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                 // next K copy whose stage is already free, else the next V copy
                 if (nk < T && nk < nv + kStages &&
                     (nk < kStages ||
-                     mbar_try(smem_u32(&st.k_empty[nk % kStages]), ((nk / kStages) - 1) & 1))) {
+                     mbar_test(smem_u32(&st.k_empty[nk % kStages]), ((nk / kStages) - 1) & 1))) {
                     load(nk++, false);
                     continue;
                 }
@@ -369,7 +389,9 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
             if (!__all_sync(0xffffffffu, mbar_wait(&st.s_full[sb], (t >> 1) & 1, abort))) { ok = false; break; }
             tc_fence_after();
             uint32_t pk[S_TOK / 2];                      // P, bf16 pairs
-            float2 ps = make_float2(0.f, 0.f);           // sum of the rounded P
+            float2 ps[4];                                // sum of the rounded P
+#pragma unroll
+            for (int k = 0; k < 4; ++k) ps[k] = make_float2(0.f, 0.f);
 
             if (t < U) {
                 const int c = s_union[t];
@@ -393,28 +415,28 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                     tmem_wait_ld();
                     if (sel) {
                         // intra-chunk softmax scaled by exp(s^_c - M0) / z_c
-                        float mx = __uint_as_float(rr[0]);
-#pragma unroll
-                        for (int j = 1; j < S_TOK; ++j) mx = fmaxf(mx, __uint_as_float(rr[j]));
+                        const float mx = row_max(rr, S_TOK);
                         const float2 nb = make_float2(-mx * sl2, -mx * sl2);
                         float2 e[S_TOK / 2];
-                        float2 z2 = make_float2(0.f, 0.f);
+                        float2 z2[4];
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) z2[k] = make_float2(0.f, 0.f);
 #pragma unroll
                         for (int j = 0; j < S_TOK / 2; ++j) {
                             e[j] = f2_fma(make_float2(__uint_as_float(rr[2 * j]),
                                                       __uint_as_float(rr[2 * j + 1])), sl2v, nb);
                             e[j].x = fast_exp2(e[j].x);
                             e[j].y = fast_exp2(e[j].y);
-                            z2 = f2_add(z2, e[j]);
+                            z2[j & 3] = f2_add(z2[j & 3], e[j]);
                         }
-                        const float f = fast_exp2(sh - M0l2) / (z2.x + z2.y);
+                        const float2 zz = f2_add(f2_add(z2[0], z2[1]), f2_add(z2[2], z2[3]));
+                        const float f = __fdividef(fast_exp2(sh - M0l2), zz.x + zz.y);
                         const float2 fv = make_float2(f, f);
 #pragma unroll
                         for (int j = 0; j < S_TOK / 2; ++j) {
                             const float2 pv = f2_mul(e[j], fv);
                             pk[j] = pack_bf16(pv.x, pv.y);
-                            ps = f2_add(ps, make_float2(__uint_as_float(pk[j] << 16),
-                                                        __uint_as_float(pk[j] & 0xffff0000u)));
+                            acc_bf16x2(ps[j & 3], pk[j]);
                         }
                     } else {
 #pragma unroll
@@ -440,10 +462,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                         rr[j] = in ? rr[j] : __float_as_uint(-INFINITY);
                     }
                 }
-                float mx = __uint_as_float(rr[0]);
-#pragma unroll
-                for (int j = 1; j < S_TOK; ++j) mx = fmaxf(mx, __uint_as_float(rr[j]));
-                mx *= sl2;                                   // log2 units
+                float mx = row_max(rr, S_TOK) * sl2;         // log2 units
                 const bool mine = mx > mref + kRescaleLog2;
                 if (__any_sync(0xffffffffu, mine)) {
                     // raise the reference max of the rows that need it and
@@ -480,8 +499,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                     e.x = fast_exp2(e.x);
                     e.y = fast_exp2(e.y);
                     pk[j] = pack_bf16(e.x, e.y);
-                    ps = f2_add(ps, make_float2(__uint_as_float(pk[j] << 16),
-                                                __uint_as_float(pk[j] & 0xffff0000u)));
+                    acc_bf16x2(ps[j & 3], pk[j]);
                 }
             }
 
@@ -492,7 +510,10 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
             // ~2^-9 w|v|.
 #pragma unroll
             for (int c0 = 0; c0 < S_TOK / 2; c0 += 32) tmem_st32(tS + c0, pk + c0);
-            l += ps.x + ps.y;
+            {
+                const float2 pt = f2_add(f2_add(ps[0], ps[1]), f2_add(ps[2], ps[3]));
+                l += pt.x + pt.y;
+            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&st.p_full[sb]);

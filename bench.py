@@ -115,6 +115,37 @@ def decode_bytes(sh, cache_len):
     return float(tot)
 
 
+def decode_multi_bytes(sh, cache_len, T, idx):
+    """Touched HBM bytes of one T-token decode step: k' and b' of every
+    candidate once per (sequence, kv head) (one shared scan), K and V of the
+    union over the T tokens of their selected chunks and windows, Q, O, idx.
+    idx is the step's [B, T, Hkv, K] selection (host array)."""
+    tot = 0
+    esz = 2 if sh.dtype == "bf16" else 4
+    for b, L in enumerate(cache_len):
+        i_last = L - 1
+        nc_last = max((i_last - sh.W + 1) // sh.S, 0)
+        tot += nc_last * sh.Hkv * (sh.d * esz + 4)
+        for g in range(sh.Hkv):
+            spans = []
+            for t in range(T):
+                i = L - T + t
+                lq = (i - sh.W + 1) // sh.S
+                spans.append((max(lq * sh.S, 0), i + 1))
+                spans += [(int(c) * sh.S, int(c) * sh.S + sh.S)
+                          for c in idx[b, t, g] if c >= 0]
+            spans.sort()
+            n, end = 0, -1
+            for a, e in spans:                   # length of the union
+                if e <= end:
+                    continue
+                n += e - max(a, end)
+                end = e
+            tot += n * 2 * sh.d * esz
+        tot += T * (2 * sh.Hq * sh.d * esz + sh.Hkv * sh.K * 4)
+    return float(tot)
+
+
 # ------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi sampling of SM clock and throttle reasons during a region."""
@@ -385,8 +416,11 @@ def main():
         flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
         d = bench_decode(args, dev, torch.cuda.current_stream(dev), flush,
                          world, max_over_ranks, barrier, rank, peaks)
+        dm = bench_decode_multi(args, dev, torch.cuda.current_stream(dev),
+                                flush, world, max_over_ranks, barrier, rank,
+                                peaks)
         if rank == 0:
-            print(json.dumps({"decode": d}), flush=True)
+            print(json.dumps({"decode": d, "decode_multi": dm}), flush=True)
         ranks.close()
         return
     inp = synth.make_prefill(sh, seed=synth.seed_for(cfg_id) + 17 * rank,
@@ -513,6 +547,9 @@ def main():
     if not args.no_decode:
         line["decode"] = bench_decode(args, dev, stream, flush, world,
                                       max_over_ranks, barrier, rank, peaks)
+        line["decode_multi"] = bench_decode_multi(
+            args, dev, stream, flush, world, max_over_ranks, barrier, rank,
+            peaks)
         line["landmarks"] = bench_landmarks(args, dev, stream, flush,
                                             max_over_ranks, barrier, peaks)
 
@@ -670,6 +707,113 @@ def bench_decode(args, dev, stream, flush, world, max_over_ranks, barrier,
     del inp, O, idx, sel, ws
     torch.cuda.empty_cache()
     return out
+
+
+DECODE_MULTI_T = 4
+
+
+def bench_decode_multi(args, dev, stream, flush, world, max_over_ranks,
+                       barrier, rank, peaks):
+    """Speculative decode: the 512K batch-8 decode workload with T = 4 query
+    tokens per sequence (positions L-4 .. L-1) in one step, as a CUDA graph,
+    L2 flushed before every timed step. HBM roofline on the bytes the step
+    must touch: one landmark scan per (sequence, kv head) and the union of
+    the T tokens' chunks and windows."""
+    import torch
+
+    import chunk_sparse_long_landmark_b200 as hils
+    import synth
+    name, cid = DECODE_WORKLOAD
+    sh = synth.DECODE_CONFIGS[cid]
+    T = DECODE_MULTI_T
+    inp = synth.make_decode(sh, seed=synth.seed_for(cid) + 17 * rank + 5,
+                            device=dev)
+    g0 = torch.Generator(device=dev).manual_seed(synth.seed_for(cid) + 29)
+    Qm = torch.randn(sh.B, T, sh.Hq, sh.d, generator=g0,
+                     device=dev).to(torch.bfloat16)
+    O = torch.empty_like(Qm)
+    idx = torch.empty(sh.B, T, sh.Hkv, sh.K, dtype=torch.int32, device=dev)
+    sel = torch.empty(sh.B, T, sh.Hq, sh.K, dtype=torch.float32, device=dev)
+    side = torch.cuda.Stream(dev)
+    ws = None
+
+    def call(st):
+        nonlocal ws
+        _, _ = hils.fwd_decode_multi(Qm, inp["K"], inp["V"], inp["Klm"],
+                                     inp["bias"], inp["cache_len"],
+                                     inp["head_map"], sh.S, sh.W, sh.K,
+                                     out=O, idx=idx, sel_score=sel,
+                                     workspace=ws, stream=st)
+
+    n = ctypes_workspace_multi(hils, Qm, inp, sh, T)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(side):
+        for _ in range(args.warmup):
+            call(side)
+    side.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        call(side)
+    torch.cuda.synchronize()
+    steps = max(args.steps, 20)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    barrier()
+    evs = [(torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    cur = torch.cuda.current_stream(dev)
+    for a, b in evs:
+        flush.zero_()
+        a.record(cur)
+        g.replay()
+        b.record(cur)
+    torch.cuda.synchronize()
+    times = [a.elapsed_time(b) for a, b in evs]
+    ms = max_over_ranks(sum(times)) / steps
+    cl = inp["cache_len"].cpu().tolist()
+    nbytes = decode_multi_bytes(sh, cl, T, idx.cpu().numpy())
+    ach = nbytes / (ms * 1e-3) / 1e9
+    del g
+    out = {
+        "workload": f"{name}_T{T}", "value": ms * 1e3, "unit": "us/step",
+        "note": f"one step = {T} speculative query tokens for each of the "
+                f"B={sh.B} sequences (positions L-{T} .. L-1)",
+        "median_us": statistics.median(times) * 1e3,
+        "tokens_per_s": world * sh.B * T / (ms * 1e-3),
+        "roofline": {"bound": "hbm", "kernel": "whole multi-token step (graph)",
+                     "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": ach / peaks["hbm"], "peak_source": peaks["src"],
+                     "algorithmic_bytes_per_step": nbytes,
+                     "bytes_model": "k', b' once per (sequence, kv head); K, V "
+                                    "of the union of the tokens' chunks and "
+                                    "windows",
+                     "traffic": None},
+        "config": {"B": sh.B, "T": T, "Hq": sh.Hq, "Hkv": sh.Hkv, "d": sh.d,
+                   "L": sh.N, "S": sh.S, "W": sh.W, "K": sh.K,
+                   "l2": "flushed before every timed step"},
+    }
+    del inp, Qm, O, idx, sel, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def ctypes_workspace_multi(hils, Qm, inp, sh, T):
+    """Workspace bytes of the multi-token step (with sel_score given)."""
+    import ctypes
+    hm = (ctypes.c_int32 * sh.Hq)(*inp["head_map"])
+    fake = 1 << 40
+    base = hils.DecodeArgs(hils.BF16, sh.B, sh.Hq, sh.Hkv, sh.N, sh.d, sh.S,
+                           sh.W, sh.K, ctypes.cast(hm, ctypes.c_void_p), fake,
+                           None, fake, fake, fake, fake, fake, fake, fake,
+                           fake, None, 0, None)
+    a = hils.DecodeMultiArgs(base, T, None, 0)
+    n = ctypes.c_size_t(0)
+    rc = hils.lib().hils_decode_multi_workspace_size(ctypes.byref(a),
+                                                     ctypes.byref(n))
+    if rc:
+        raise hils.HilsError(rc, "hils_decode_multi_workspace_size")
+    return max(n.value, 1)
 
 
 if __name__ == "__main__":

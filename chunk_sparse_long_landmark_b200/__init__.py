@@ -20,6 +20,7 @@ __all__ = [
     "decode_workspace_size", "PrefillArgs", "DecodeArgs", "STATUS",
     "launch_count", "fwd_decode_noalloc", "build_landmarks", "LandmarkArgs",
     "chunk_overlap", "fwd_decode_paged", "DecodePagedArgs",
+    "fwd_decode_multi", "DecodeMultiArgs",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -41,6 +42,7 @@ symbols = [
     "hils_decode_attend", "hils_launch_count", "hils_fwd_decode_noalloc",
     "hils_build_landmarks", "hils_chunk_overlap",
     "hils_decode_paged_workspace_size", "hils_fwd_decode_paged",
+    "hils_decode_multi_workspace_size", "hils_fwd_decode_multi",
 ]
 
 
@@ -74,6 +76,11 @@ class DecodeArgs(ctypes.Structure):
 
 class DecodePagedArgs(ctypes.Structure):
     _fields_ = [("base", DecodeArgs), ("block_table", _p), ("n_pages", _i)]
+
+
+class DecodeMultiArgs(ctypes.Structure):
+    _fields_ = [("base", DecodeArgs), ("T", _i), ("block_table", _p),
+                ("n_pages", _i)]
 
 
 class LandmarkArgs(ctypes.Structure):
@@ -120,6 +127,12 @@ def lib():
                 ctypes.POINTER(DecodePagedArgs), ctypes.POINTER(ctypes.c_size_t)]
             L.hils_fwd_decode_paged.restype = ctypes.c_int
             L.hils_fwd_decode_paged.argtypes = [ctypes.POINTER(DecodePagedArgs),
+                                                ctypes.c_void_p]
+            L.hils_decode_multi_workspace_size.restype = ctypes.c_int
+            L.hils_decode_multi_workspace_size.argtypes = [
+                ctypes.POINTER(DecodeMultiArgs), ctypes.POINTER(ctypes.c_size_t)]
+            L.hils_fwd_decode_multi.restype = ctypes.c_int
+            L.hils_fwd_decode_multi.argtypes = [ctypes.POINTER(DecodeMultiArgs),
                                                 ctypes.c_void_p]
             L.hils_chunk_overlap.restype = ctypes.c_int
             L.hils_chunk_overlap.argtypes = [_p] + [_i] * 6 + [_p] * 4
@@ -404,4 +417,60 @@ def fwd_decode_paged(Q, Kpool, Vpool, Klm, bias, cache_len, block_table,
     rc = lib().hils_fwd_decode_paged(ctypes.byref(a), _stream_handle(stream))
     if rc:
         raise HilsError(rc, "hils_fwd_decode_paged")
+    return out, idx
+
+
+def fwd_decode_multi(Q, Kc, V, Klm, bias, cache_len, head_map, S, W, topk,
+                     block_table=None, Qs=None, out=None, idx=None,
+                     sel_score=None, workspace=None, status=None,
+                     stream=None):
+    """Multi-token (speculative) decode through hils_fwd_decode_multi.
+    Returns (O, idx).
+
+    Q [B,T,Hq,d] (token-major): token t of sequence b sits at position
+    cache_len[b]-T+t. Kc/V [B,Hkv,Lmax,d], or the page pool [n_pages,Hkv,S,d]
+    when block_table (int32 [B, Lmax//S], device) is given. Klm
+    [B,Hkv,Lmax//S,d], bias [B,Hkv,Lmax//S], cache_len int32 [B] on the
+    device. O [B,T,Hq,d], idx [B,T,Hkv,topk]."""
+    import torch
+    _dev(Q, Kc, V, Klm, bias, cache_len, block_table, Qs, out, idx,
+         sel_score, workspace, status)
+    B, T, Hq, d = Q.shape
+    Hkv = Kc.shape[1]
+    if block_table is not None:
+        if block_table.dtype != torch.int32 or not block_table.is_contiguous():
+            raise ValueError("block_table must be a contiguous int32 tensor")
+        Lmax = block_table.shape[1] * S
+        n_pages = Kc.shape[0]
+    else:
+        Lmax = Kc.shape[2]
+        n_pages = 0
+    hm = _head_map_array(head_map, Hq)
+    if out is None:
+        out = torch.empty_like(Q)
+    if idx is None:
+        idx = torch.empty(B, T, Hkv, topk, dtype=torch.int32, device=Q.device)
+
+    def record(ws):
+        base = DecodeArgs(_dtype_code(Q), B, Hq, Hkv, Lmax, d, S, W, topk,
+                          ctypes.cast(hm, ctypes.c_void_p), _ptr(Q), _ptr(Qs),
+                          _ptr(Kc), _ptr(V), _ptr(Klm), _ptr(bias),
+                          _ptr(cache_len), _ptr(out), _ptr(idx),
+                          _ptr(sel_score), _ptr(ws),
+                          0 if ws is None else ws.numel() * ws.element_size(),
+                          _ptr(status))
+        return DecodeMultiArgs(base, T, _ptr(block_table), n_pages)
+
+    if workspace is None:
+        n = ctypes.c_size_t(0)
+        rc = lib().hils_decode_multi_workspace_size(ctypes.byref(record(None)),
+                                                    ctypes.byref(n))
+        if rc:
+            raise HilsError(rc, "hils_decode_multi_workspace_size")
+        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8,
+                                device=Q.device)
+    a = record(workspace)
+    rc = lib().hils_fwd_decode_multi(ctypes.byref(a), _stream_handle(stream))
+    if rc:
+        raise HilsError(rc, "hils_fwd_decode_multi")
     return out, idx

@@ -21,6 +21,14 @@
 //               tiles), merged online -> partial (m, l, o) per group; the
 //               CTA that arrives last for its (b, kv head) combines the
 //               partials in group order (deterministic) and writes O.
+//
+// Multi-token (speculative) decode, Sec. 4.2 / Sec. 7.1: T query tokens per
+// sequence at positions cache_len-T .. cache_len-1, token-major ([B, T, H,
+// ...] = [B*T, H, ...]). dec_score scans each landmark tile once for all T x
+// G queries of a (b, kv head) (the T tokens are extra columns of the same
+// MMA); dec_select and dec_attend then run per (token, kv head) -- a
+// "virtual sequence" v = b*T + t -- reading the physical cache of b. T = 1
+// is plain decode.
 #include <math.h>
 
 #include "hils_fast.cuh"
@@ -49,12 +57,13 @@ struct DecParams {
     int32_t *idx;
     float *sel;
     int32_t *status;
-    float *ws_s;        // [B, Hkv, G, ncs] raw s^
-    float *ws_p;        // [B, Hkv, nsplit, G, 2] (max, sum exp(s^ - max))
-    float *ws_o;        // [B, Hkv, ntile, G, d] partial outputs
-    float *ws_ml;       // [B, Hkv, ntile, G, 2] partial (m, l)
-    int32_t *ws_cnt;    // [B, Hkv] arrival tickets
+    float *ws_s;        // [B, Hkv, T, G, ncs] raw s^
+    float *ws_p;        // [B, Hkv, T, nsplit, G, 2] (max, sum exp(s^ - max))
+    float *ws_o;        // [B*T, Hkv, ntile, G, d] partial outputs
+    float *ws_ml;       // [B*T, Hkv, ntile, G, 2] partial (m, l)
+    int32_t *ws_cnt;    // [B*T, Hkv] arrival tickets
     int B, Hq, Hkv, G, d, S, W, K, Lmax, nC;
+    int T;              // query tokens per sequence (1: plain decode)
     int ncs;            // chunk stride of ws_s (max candidates of any row)
     int nsplit;         // landmark splits per (b, g)
     int cps;            // chunks per split (multiple of kTileChunks)
@@ -99,17 +108,20 @@ __device__ __forceinline__ uint32_t swz(int r, int u) {
     return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4));
 }
 
-__device__ __forceinline__ bool seq_ok(const DecParams &p, int b, int64_t *i,
-                                       int64_t *w0, int64_t *nc) {
+// Position of token `tok` (0..T-1) of sequence b: cache_len[b] - T + tok.
+// False when cache_len[b] is outside [T, Lmax].
+__device__ __forceinline__ bool tok_ok(const DecParams &p, int b, int tok,
+                                       int64_t *i, int64_t *w0, int64_t *nc) {
     const int L = p.cache_len[b];
-    if (L < 1 || L > p.Lmax) return false;
-    *i = L - 1;
+    if (L < p.T || L > p.Lmax) return false;
+    *i = (int64_t)L - p.T + tok;
     window_bounds(*i, p.S, p.W, w0, nc);
     return true;
 }
 
 // --------------------------------------------------------------- dec_score
-template <int D>
+// NG column groups of 8: column n = token * G + head slot (n < T*G <= 8*NG).
+template <int D, int NG>
 __global__ void __launch_bounds__(kScoreWarps * 32)
 dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
     constexpr int HALVES = D / 64;
@@ -117,16 +129,17 @@ dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     __shared__ uint64_t full[kScoreStages];
-    __shared__ float red_m[kScoreWarps][8], red_s[kScoreWarps][8];
+    __shared__ float red_m[kScoreWarps][8 * NG], red_s[kScoreWarps][8 * NG];
 
     const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gi = lane >> 2, t = lane & 3;
-    const int G = p.G;
+    const int G = p.G, T = p.T, ncol = T * G;
     const int bg = b * p.Hkv + g;
-    if (split == 0 && threadIdx.x == 0) p.ws_cnt[bg] = 0;   // tickets of dec_attend
+    if (split == 0 && threadIdx.x < T)           // tickets of dec_attend
+        p.ws_cnt[((int64_t)b * T + threadIdx.x) * p.Hkv + g] = 0;
     int64_t i, w0, nc;
-    const bool ok = seq_ok(p, b, &i, &w0, &nc);
+    const bool ok = tok_ok(p, b, T - 1, &i, &w0, &nc);   // the last token's nc is the largest
     if (!ok) {
         if (split == 0 && threadIdx.x == 0) report(p.status, HILS_ERR_DEVICE_BAD_LENGTH);
         return;
@@ -135,20 +148,37 @@ dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
     const int c_end = (int)min((int64_t)c_begin + p.cps, nc);
     const int ntiles = c_end > c_begin ? (c_end - c_begin + kTileChunks - 1) / kTileChunks : 0;
 
-    // scoring query as the B operand: column n = head slot gi (< G), rows = dims
+    // scoring queries as the B operand: column n = (token, head slot), rows = dims
     const void *qb = p.Qs ? p.Qs : p.Q;
-    uint32_t bq[D / 16][2];
+    uint32_t bq[NG][D / 16][2];
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-        bq[ks][0] = bq[ks][1] = 0u;
-        if (gi < G) {
-            const int h = p.group_heads[g * G + gi];
-            const uint32_t *q = reinterpret_cast<const uint32_t *>(
-                reinterpret_cast<const __nv_bfloat16 *>(qb) + ((int64_t)b * p.Hq + h) * D);
-            bq[ks][0] = q[(ks * 16 + 2 * t) >> 1];
-            bq[ks][1] = q[(ks * 16 + 8 + 2 * t) >> 1];
+    for (int ng = 0; ng < NG; ++ng) {
+        const int n = ng * 8 + gi;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            bq[ng][ks][0] = bq[ng][ks][1] = 0u;
+            if (n < ncol) {
+                const int h = p.group_heads[g * G + n % G];
+                const uint32_t *q = reinterpret_cast<const uint32_t *>(
+                    reinterpret_cast<const __nv_bfloat16 *>(qb) +
+                    (((int64_t)b * T + n / G) * p.Hq + h) * D);
+                bq[ng][ks][0] = q[(ks * 16 + 2 * t) >> 1];
+                bq[ng][ks][1] = q[(ks * 16 + 8 + 2 * t) >> 1];
+            }
         }
     }
+    // candidates of this lane's output columns 8 ng + 2t + k (token of the
+    // column): a token before the last may have fewer
+    int nc_col[NG][2];
+#pragma unroll
+    for (int ng = 0; ng < NG; ++ng)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int n = ng * 8 + 2 * t + k;
+            int64_t ii, ww, nn = 0;
+            if (n < ncol) tok_ok(p, b, n / G, &ii, &ww, &nn);
+            nc_col[ng][k] = (int)nn;
+        }
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kScoreStages; ++s) mbar_init(&full[s], 1);
@@ -164,11 +194,15 @@ dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
                             &full[tt], hf * 64, (int)(row0 + tt * kTileChunks));
         }
     }
-    // per lane: heads 2t, 2t+1 (when < G); running max / sum in log2 units
-    float mx[2] = {-INFINITY, -INFINITY}, sm[2] = {0.f, 0.f};
+    // per lane: columns 8 ng + 2t, +1 (when < T*G); running max / sum, log2 units
+    float mx[NG][2], sm[NG][2];
+#pragma unroll
+    for (int ng = 0; ng < NG; ++ng)
+        mx[ng][0] = mx[ng][1] = -INFINITY, sm[ng][0] = sm[ng][1] = 0.f;
     const float sl2 = p.inv_sqrt_d * kLog2e;
     const float *bias = p.bias + (int64_t)bg * p.nC;
-    float *outs = p.ws_s + (int64_t)bg * G * p.ncs;
+    // s^ of column n = (token, head slot) at ((bg * T + token) * G + slot) * ncs
+    float *outs = p.ws_s + (int64_t)bg * T * G * p.ncs;
     volatile int dummy_abort = 0;
     // bias of the lane's 2 chunks of the next tile, loaded a tile ahead
     auto load_bias = [&](int tt, float *bv) {
@@ -185,7 +219,9 @@ dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
         const float bcur[2] = {bnext[0], bnext[1]};
         load_bias(tt + 1, bnext);
         mbar_wait(&full[s], (tt / kScoreStages) & 1, &dummy_abort);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        float acc[NG][4];
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng) acc[ng][0] = acc[ng][1] = acc[ng][2] = acc[ng][3] = 0.f;
         const uint32_t base = smem_u32(smem + s * STAGE);
         const int r = warp * 16 + (lane & 15);
 #pragma unroll
@@ -193,7 +229,9 @@ dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
             const int hf = ks / 4, u = (ks % 4) * 2 + (lane >> 4);
             uint32_t a[4];
             ldsm_x4(base + hf * (kTileChunks * 128) + swz(r, u), a);
-            mma_bf16(acc, a, bq[ks][0], bq[ks][1]);
+#pragma unroll
+            for (int ng = 0; ng < NG; ++ng)
+                if (ng * 8 < ncol) mma_bf16(acc[ng], a, bq[ng][ks][0], bq[ng][ks][1]);
         }
         __syncthreads();                         // stage s fully read
         if (threadIdx.x == 0 && tt + kScoreStages < ntiles) {
@@ -203,20 +241,28 @@ dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
                 tma_load_2d(smem + s * STAGE + hf * (kTileChunks * 128), &tmL,
                             &full[s], hf * 64, (int)(row0 + tn * kTileChunks));
         }
-        // acc: chunks (gi, gi+8) of this warp's 16, heads (2t, 2t+1)
+        // acc[ng]: chunks (gi, gi+8) of this warp's 16, columns 8 ng + (2t, 2t+1)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int hh = 2 * t + (q & 1);
-            const int c = c_begin + tt * kTileChunks + warp * 16 + gi + (q >> 1) * 8;
-            if (hh < G && c < c_end) {
-                const float shat = fmaf(acc[q], p.inv_sqrt_d, bcur[q >> 1]);
-                outs[(int64_t)hh * p.ncs + c] = shat;
-                const float x = shat * kLog2e;
+        for (int ng = 0; ng < NG; ++ng)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int n = ng * 8 + 2 * t + (q & 1);
                 const int k = q & 1;
-                if (x > mx[k]) { sm[k] = sm[k] * fast_exp2(mx[k] - x) + 1.f; mx[k] = x; }
-                else sm[k] += fast_exp2(x - mx[k]);
+                const int c = c_begin + tt * kTileChunks + warp * 16 + gi + (q >> 1) * 8;
+                if (n < ncol && c < c_end) {
+                    const float shat = fmaf(acc[ng][q], p.inv_sqrt_d, bcur[q >> 1]);
+                    outs[(int64_t)n * p.ncs + c] = shat;
+                    if (c < nc_col[ng][k]) {
+                        const float x = shat * kLog2e;
+                        if (x > mx[ng][k]) {
+                            sm[ng][k] = sm[ng][k] * fast_exp2(mx[ng][k] - x) + 1.f;
+                            mx[ng][k] = x;
+                        } else {
+                            sm[ng][k] += fast_exp2(x - mx[ng][k]);
+                        }
+                    }
+                }
             }
-        }
     }
     (void)sl2;
     grid_dep_launch();                           // dec_select may start now
@@ -231,31 +277,34 @@ dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
     }
     // reduce (max, sum) over the 8 chunk lanes (gi) then over warps
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-        for (int o = 4; o < 32; o <<= 1) {
-            const float om = __shfl_xor_sync(0xffffffffu, mx[k], o);
-            const float os = __shfl_xor_sync(0xffffffffu, sm[k], o);
-            const float mn = fmaxf(mx[k], om);
-            sm[k] = (mn == -INFINITY) ? 0.f
-                    : sm[k] * fast_exp2(mx[k] - mn) + os * fast_exp2(om - mn);
-            mx[k] = mn;
+    for (int ng = 0; ng < NG; ++ng)
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            for (int o = 4; o < 32; o <<= 1) {
+                const float om = __shfl_xor_sync(0xffffffffu, mx[ng][k], o);
+                const float os = __shfl_xor_sync(0xffffffffu, sm[ng][k], o);
+                const float mn = fmaxf(mx[ng][k], om);
+                sm[ng][k] = (mn == -INFINITY) ? 0.f
+                            : sm[ng][k] * fast_exp2(mx[ng][k] - mn) + os * fast_exp2(om - mn);
+                mx[ng][k] = mn;
+            }
+            if (gi == 0) {
+                red_m[warp][ng * 8 + 2 * t + k] = mx[ng][k];
+                red_s[warp][ng * 8 + 2 * t + k] = sm[ng][k];
+            }
         }
-    }
-    if (gi == 0) {
-        red_m[warp][2 * t] = mx[0]; red_s[warp][2 * t] = sm[0];
-        red_m[warp][2 * t + 1] = mx[1]; red_s[warp][2 * t + 1] = sm[1];
-    }
     __syncthreads();
-    if (threadIdx.x < G) {
-        const int hh = threadIdx.x;
+    if (threadIdx.x < ncol) {
+        const int n = threadIdx.x;
         float m = -INFINITY, s2 = 0.f;
         for (int w = 0; w < kScoreWarps; ++w) {
-            const float om = red_m[w][hh], os = red_s[w][hh];
+            const float om = red_m[w][n], os = red_s[w][n];
             const float mn = fmaxf(m, om);
             s2 = (mn == -INFINITY) ? 0.f : s2 * fast_exp2(m - mn) + os * fast_exp2(om - mn);
             m = mn;
         }
-        float *pp = p.ws_p + (((int64_t)bg * p.nsplit + split) * G + hh) * 2;
+        // partials of (b, g, token) at ((bg * T + token) * nsplit + split) * G + slot
+        float *pp = p.ws_p + ((((int64_t)bg * T + n / G) * p.nsplit + split) * G + n % G) * 2;
         pp[0] = m;          // log2 units
         pp[1] = s2;
     }
@@ -311,13 +360,16 @@ dec_select_kernel(const DecParams p) {
     __shared__ int ncand;
     __shared__ uint32_t cand_k[kCandCap];
     __shared__ int cand_c[kCandCap];
-    const int g = blockIdx.x, b = blockIdx.y;
-    const int bg = b * p.Hkv + g;
+    // one CTA per (token v = b*T + tok, kv head g)
+    const int g = blockIdx.x, v = blockIdx.y;
+    const int b = v / p.T, tok = v - b * p.T;
+    const int bgt = (b * p.Hkv + g) * p.T + tok;     // score workspace row
+    const int bgv = v * p.Hkv + g;                   // idx row
     const int G = p.G, K = p.K;
     int64_t i, w0, nc64;
-    if (!seq_ok(p, b, &i, &w0, &nc64)) return;
+    if (!tok_ok(p, b, tok, &i, &w0, &nc64)) return;
     const int nc = (int)nc64;
-    const float *ss = p.ws_s + (int64_t)bg * G * p.ncs;
+    const float *ss = p.ws_s + (int64_t)bgt * G * p.ncs;
     grid_dep_wait();                             // dec_score's s^ and partials
     grid_dep_launch();                           // dec_attend may start now
 
@@ -326,7 +378,7 @@ dec_select_kernel(const DecParams p) {
     const int nsp = (nc + p.cps - 1) / p.cps;
     const bool staged = nsp * G <= kSelThreads && nsp <= kMaxSplits;
     if (staged && threadIdx.x < nsp * G) {
-        const float *pp = p.ws_p + ((int64_t)bg * p.nsplit * G + threadIdx.x) * 2;
+        const float *pp = p.ws_p + ((int64_t)bgt * p.nsplit * G + threadIdx.x) * 2;
         part[threadIdx.x][0] = pp[0];
         part[threadIdx.x][1] = pp[1];
     }
@@ -336,7 +388,7 @@ dec_select_kernel(const DecParams p) {
         float m = -INFINITY, s2 = 0.f;
         for (int sp = 0; sp < nsp; ++sp) {
             const float *pp = staged ? part[sp * G + hh]
-                                     : p.ws_p + (((int64_t)bg * p.nsplit + sp) * G + hh) * 2;
+                                     : p.ws_p + (((int64_t)bgt * p.nsplit + sp) * G + hh) * 2;
             const float om = pp[0], os = pp[1];
             const float mn = fmaxf(m, om);
             s2 = (mn == -INFINITY) ? 0.f : s2 * exp2f(m - mn) + os * exp2f(om - mn);
@@ -448,10 +500,10 @@ dec_select_kernel(const DecParams p) {
             if (mine) {                          // ascending chunk order
                 int pos = 0;
                 for (int f = 0; f < m; ++f) pos += (cand_k[f] && cand_c[f] < mc) ? 1 : 0;
-                p.idx[(int64_t)bg * K + pos] = mc;
+                p.idx[(int64_t)bgv * K + pos] = mc;
                 for (int hh = 0; hh < G; ++hh) {
                     const int h = p.group_heads[g * G + hh];
-                    p.sel[((int64_t)b * p.Hq + h) * K + pos] = ss[(int64_t)hh * p.ncs + mc];
+                    p.sel[((int64_t)v * p.Hq + h) * K + pos] = ss[(int64_t)hh * p.ncs + mc];
                 }
             }
             return;                              // nc > K: no padding
@@ -532,19 +584,19 @@ dec_select_kernel(const DecParams p) {
         selbits &= selbits - 1;
         const int c = cbeg + q;
         if (pos < K) {
-            p.idx[(int64_t)bg * K + pos] = c;
+            p.idx[(int64_t)bgv * K + pos] = c;
             for (int hh = 0; hh < G; ++hh) {
                 const int h = p.group_heads[g * G + hh];
-                p.sel[((int64_t)b * p.Hq + h) * K + pos] = ss[(int64_t)hh * p.ncs + c];
+                p.sel[((int64_t)v * p.Hq + h) * K + pos] = ss[(int64_t)hh * p.ncs + c];
             }
         }
         ++pos;
     }
     for (int k = nsel + threadIdx.x; k < K; k += kSelThreads) {
-        p.idx[(int64_t)bg * K + k] = -1;
+        p.idx[(int64_t)bgv * K + k] = -1;
         for (int hh = 0; hh < G; ++hh) {
             const int h = p.group_heads[g * G + hh];
-            p.sel[((int64_t)b * p.Hq + h) * K + k] = __int_as_float(0x7fc00000);
+            p.sel[((int64_t)v * p.Hq + h) * K + k] = __int_as_float(0x7fc00000);
         }
     }
 }
@@ -578,13 +630,17 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     // every copy has landed and been read, so it shares the stage buffers
     float *ored = reinterpret_cast<float *>(smem);
 
-    const int grp = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int bg = b * p.Hkv + g;
+    // (token v = b*T + tok, kv head g): cache rows of sequence b, everything
+    // else (Q, idx, s^, O, partials, tickets) of the token
+    const int grp = blockIdx.x, g = blockIdx.y, v = blockIdx.z;
+    const int b = v / p.T, tok = v - b * p.T;
+    const int bgc = b * p.Hkv + g;                   // cache rows
+    const int bg = v * p.Hkv + g;                    // the token's rows
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gi = lane >> 2, t = lane & 3;
     const int G = p.G;
     int64_t i = 0, w0 = 0, nc = 0;
-    const bool ok = seq_ok(p, b, &i, &w0, &nc);
+    const bool ok = tok_ok(p, b, tok, &i, &w0, &nc);
     // the selection always holds min(|C_i|, K) chunks, so the tile list is
     // known before the selection itself is read
     const int nsel = ok ? (int)min(nc, (int64_t)p.K) : 0;
@@ -609,7 +665,7 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     // [n_pages,Hkv,S,d] (a tile is one chunk, i.e. one page)
     auto tile_row = [&](int tau) -> int64_t {
         const int64_t j0 = tile_j0(tau);
-        if (!p.block_table) return (int64_t)bg * p.Lmax + j0;
+        if (!p.block_table) return (int64_t)bgc * p.Lmax + j0;
         const int pg = p.block_table[(int64_t)b * (p.Lmax / p.S) + j0 / p.S];
         if (pg < 0 || pg >= p.n_pages) {         // a box wholly before row 0:
             report(p.status, HILS_ERR_DEVICE_BAD_LENGTH);   // TMA reads zeros
@@ -640,7 +696,7 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     for (int e = threadIdx.x; e < G * p.K; e += kAttThreads) {
         const int hh = e / p.K, kk = e % p.K;
         const int h = p.group_heads[g * G + hh];
-        s_sel[e] = ok ? p.sel[((int64_t)b * p.Hq + h) * p.K + kk] : 0.f;
+        s_sel[e] = ok ? p.sel[((int64_t)v * p.Hq + h) * p.K + kk] : 0.f;
     }
     __syncthreads();
     if (threadIdx.x == 0)
@@ -656,7 +712,7 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
             if (gi < G) {
                 const int h = p.group_heads[g * G + gi];
                 const uint32_t *q = reinterpret_cast<const uint32_t *>(
-                    reinterpret_cast<const __nv_bfloat16 *>(p.Q) + ((int64_t)b * p.Hq + h) * D);
+                    reinterpret_cast<const __nv_bfloat16 *>(p.Q) + ((int64_t)v * p.Hq + h) * D);
                 aq[ks][0] = q[(ks * 16 + 2 * t) >> 1];
                 aq[ks][2] = q[(ks * 16 + 8 + 2 * t) >> 1];
             }
@@ -865,7 +921,7 @@ dec_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                 if (g0 + u < ngrp) num += cw[(g0 + u) * G + hh] * v[u];
         }
         const int h = p.group_heads[g * G + hh];
-        reinterpret_cast<__nv_bfloat16 *>(p.O)[((int64_t)b * p.Hq + h) * D + c] =
+        reinterpret_cast<__nv_bfloat16 *>(p.O)[((int64_t)v * p.Hq + h) * D + c] =
             __float2bfloat16_rn(num);
     }
     if (threadIdx.x == 0) p.ws_cnt[bg] = 0;      // ready for the next call
@@ -910,7 +966,8 @@ DecPlan dec_plan(const Problem &p) {
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // one wave: at most 3 resident CTAs per SM (65 KB of stages each)
+    // one wave: at most 3 resident CTAs per SM (65 KB of stages each); the
+    // T tokens of a sequence share its scan
     const int64_t want = (int64_t)3 * sms;
     int64_t per_bg = want / ((int64_t)p.B * p.Hkv);
     if (per_bg < 1) per_bg = 1;
@@ -924,14 +981,14 @@ DecPlan dec_plan(const Problem &p) {
     // 3 shorter ones), 1 at S = 128
     {
         const int64_t slots = (int64_t)sms * (p.S == 64 ? 2 : 1);
-        int64_t groups = slots / ((int64_t)p.B * p.Hkv);
+        int64_t groups = slots / ((int64_t)p.B * p.T * p.Hkv);
         if (groups < 1) groups = 1;
         int per = (int)((pl.ntile + groups - 1) / groups);
         if (per < kAttPerMin) per = kAttPerMin;
         pl.att_per = per;
     }
     auto al = [](size_t x) { return (x + 255) / 256 * 256; };
-    const size_t bg = (size_t)p.B * p.Hkv;
+    const size_t bg = (size_t)p.B * p.T * p.Hkv;
     pl.off_s = 0;
     pl.off_p = al(pl.off_s + sizeof(float) * bg * p.G * pl.ncs);
     pl.off_o = al(pl.off_p + sizeof(float) * bg * pl.nsplit * p.G * 2);
@@ -954,7 +1011,7 @@ DecParams dec_params(const Problem &p, void *ws) {
     d.ws_ml = (float *)(base + pl.off_ml);
     d.ws_cnt = (int32_t *)(base + pl.off_cnt);
     d.B = p.B; d.Hq = p.Hq; d.Hkv = p.Hkv; d.G = p.G; d.d = p.d; d.S = p.S;
-    d.W = p.W; d.K = p.K; d.Lmax = p.kv_rows; d.nC = p.nC;
+    d.W = p.W; d.K = p.K; d.Lmax = p.kv_rows; d.nC = p.nC; d.T = p.T;
     d.ncs = pl.ncs; d.nsplit = pl.nsplit; d.cps = pl.cps; d.ntile = pl.ntile;
     d.att_per = pl.att_per;
     d.inv_sqrt_d = p.inv_sqrt_d;
@@ -987,6 +1044,7 @@ bool dec_fast_supported(const Problem &p) {
     if (!p.decode || p.dtype != HILS_BF16) return false;
     if (!(p.d == 64 || p.d == 128) || !(p.S == 64 || p.S == 128)) return false;
     if (p.G > 8 || p.nC < 1) return false;
+    if (p.T < 1 || p.T * p.G > 32) return false;
     int64_t w0, ncm;
     window_bounds((int64_t)p.kv_rows - 1, p.S, p.W, &w0, &ncm);
     if (ncm > (int64_t)kSelPer * kSelThreads) return false;
@@ -996,6 +1054,17 @@ bool dec_fast_supported(const Problem &p) {
 
 size_t dec_workspace_bytes(const Problem &p) { return dec_plan(p).total; }
 
+template <int D, int NG>
+cudaError_t launch_score_t(dim3 grid, size_t smem, cudaStream_t st,
+                           const CUtensorMap &tl, const DecParams &d) {
+    cudaError_t e = cudaFuncSetAttribute(dec_score_kernel<D, NG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    dec_score_kernel<D, NG><<<grid, kScoreWarps * 32, smem, st>>>(tl, d);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_dec_select(Problem &p, void *ws, cudaStream_t st) {
     DecParams d = dec_params(p, ws);
     CUtensorMap tl;
@@ -1003,22 +1072,19 @@ cudaError_t launch_dec_select(Problem &p, void *ws, cudaStream_t st) {
         return cudaErrorInvalidValue;
     const size_t smem = 1024 + (size_t)kScoreStages * kTileChunks * p.d * 2;
     dim3 grid(d.nsplit, p.Hkv, p.B);
+    const int ncol = p.T * p.G;
     cudaError_t e;
     if (p.d == 128) {
-        e = cudaFuncSetAttribute(dec_score_kernel<128>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess)
-            dec_score_kernel<128><<<grid, kScoreWarps * 32, smem, st>>>(tl, d);
+        if (ncol <= 8) e = launch_score_t<128, 1>(grid, smem, st, tl, d);
+        else if (ncol <= 16) e = launch_score_t<128, 2>(grid, smem, st, tl, d);
+        else e = launch_score_t<128, 4>(grid, smem, st, tl, d);
     } else {
-        e = cudaFuncSetAttribute(dec_score_kernel<64>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e == cudaSuccess)
-            dec_score_kernel<64><<<grid, kScoreWarps * 32, smem, st>>>(tl, d);
+        if (ncol <= 8) e = launch_score_t<64, 1>(grid, smem, st, tl, d);
+        else if (ncol <= 16) e = launch_score_t<64, 2>(grid, smem, st, tl, d);
+        else e = launch_score_t<64, 4>(grid, smem, st, tl, d);
     }
     if (e != cudaSuccess) return e;
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    e = launch_dependent(dec_select_kernel, dim3(p.Hkv, p.B), dim3(kSelThreads), 0, st, d);
+    e = launch_dependent(dec_select_kernel, dim3(p.Hkv, p.B * p.T), dim3(kSelThreads), 0, st, d);
     count_launches(2);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
@@ -1033,7 +1099,7 @@ cudaError_t launch_att_t(const DecParams &d, const CUtensorMap &tk,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const int ngrp = (d.ntile + d.att_per - 1) / d.att_per;
-    e = launch_dependent(dec_attend_kernel<S_TOK, D>, dim3(ngrp, d.Hkv, d.B),
+    e = launch_dependent(dec_attend_kernel<S_TOK, D>, dim3(ngrp, d.Hkv, d.B * d.T),
                          dim3(kAttThreads), smem, st, tk, tv, d);
     return e != cudaSuccess ? e : cudaGetLastError();
 }

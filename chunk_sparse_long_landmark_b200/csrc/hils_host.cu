@@ -86,6 +86,7 @@ hils_status prefill_problem(const hils_prefill_args *a, Problem *p,
                                  a->S, a->W, a->K, a->head_map, p);
     if (s != HILS_OK) return s;
     p->n_query = a->N;
+    p->T = 1;
     p->kv_rows = a->N;
     p->nC = a->N / a->S;
     p->decode = 0;
@@ -112,6 +113,7 @@ hils_status decode_problem(const hils_decode_args *a, Problem *p,
                                  a->S, a->W, a->K, a->head_map, p);
     if (s != HILS_OK) return s;
     p->n_query = 1;
+    p->T = 1;
     p->kv_rows = a->Lmax;
     p->nC = a->Lmax / a->S;
     p->decode = 1;
@@ -206,6 +208,29 @@ hils_status paged_problem(const hils_decode_paged_args *a, Problem *p,
     if (need_ptrs && !a->block_table) return HILS_ERR_INVALID_ARG;
     p->block_table = a->block_table;
     p->n_pages = a->n_pages;
+    if (!fast_path_supported(*p) || !fast_select_supported(*p))
+        return HILS_ERR_UNSUPPORTED;
+    return HILS_OK;
+}
+
+// The multi-token record: T query tokens per sequence (token-major Q, O,
+// idx, sel_score), optionally over a paged cache; HBM decode kernels only.
+hils_status multi_problem(const hils_decode_multi_args *a, Problem *p,
+                          bool need_ptrs) {
+    if (!a) return HILS_ERR_INVALID_ARG;
+    hils_status s = decode_problem(&a->base, p, need_ptrs);
+    if (s != HILS_OK) return s;
+    if (a->T < 1 || a->T > a->base.Lmax) return HILS_ERR_INVALID_ARG;
+    if (a->T * p->G > 32) return HILS_ERR_UNSUPPORTED;
+    p->T = a->T;
+    p->n_query = a->T;
+    if (a->block_table) {
+        if (a->base.Lmax % a->base.S != 0 || a->n_pages < 1) return HILS_ERR_INVALID_ARG;
+        if ((int64_t)a->n_pages * a->base.Hkv * a->base.S >= (1ll << 31))
+            return HILS_ERR_UNSUPPORTED;
+        p->block_table = a->block_table;
+        p->n_pages = a->n_pages;
+    }
     if (!fast_path_supported(*p) || !fast_select_supported(*p))
         return HILS_ERR_UNSUPPORTED;
     return HILS_OK;
@@ -313,6 +338,28 @@ hils_status hils_decode_paged_workspace_size(const hils_decode_paged_args *args,
 hils_status hils_fwd_decode_paged(const hils_decode_paged_args *args, void *stream) {
     Problem p;
     hils_status s = paged_problem(args, &p, true);
+    if (s != HILS_OK) return s;
+    Plan pl;
+    plan_workspace(p, args->base.sel_score != nullptr, &pl);
+    return run(p, pl, args->base.workspace, args->base.workspace_bytes,
+               (cudaStream_t)stream, kBoth);
+}
+
+hils_status hils_decode_multi_workspace_size(const hils_decode_multi_args *args,
+                                             size_t *bytes) {
+    if (!bytes) return HILS_ERR_INVALID_ARG;
+    Problem p;
+    hils_status s = multi_problem(args, &p, false);
+    if (s != HILS_OK) return s;
+    Plan pl;
+    plan_workspace(p, args->base.sel_score != nullptr, &pl);
+    *bytes = pl.total;
+    return HILS_OK;
+}
+
+hils_status hils_fwd_decode_multi(const hils_decode_multi_args *args, void *stream) {
+    Problem p;
+    hils_status s = multi_problem(args, &p, true);
     if (s != HILS_OK) return s;
     Plan pl;
     plan_workspace(p, args->base.sel_score != nullptr, &pl);

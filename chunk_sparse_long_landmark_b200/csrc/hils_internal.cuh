@@ -26,7 +26,8 @@ struct Problem {
     int n_pages;                 // pages of S tokens in the pool (paged only)
     int32_t *status;             // nullable
     int B, Hq, Hkv, G, d, S, W, K;
-    int n_query;                 // query rows per (b, h): N or 1
+    int n_query;                 // query rows per (b, h): N, or T (decode)
+    int T;                       // decode: query tokens per sequence (1: plain)
     int kv_rows;                 // token rows per (b, g): N or Lmax
     int nC;                      // landmark rows per (b, g)
     int decode;                  // 1: position from cache_len

@@ -236,6 +236,38 @@ hils_status hils_decode_paged_workspace_size(const hils_decode_paged_args *args,
 hils_status hils_fwd_decode_paged(const hils_decode_paged_args *args, void *stream);
 
 /*
+ * Multi-token (speculative) decode: T query tokens per sequence, at
+ * positions cache_len[b]-T .. cache_len[b]-1, whose keys and values are
+ * already in the cache ("Hierarchical Sparse Attention Done Right", Sec. 4.2:
+ * adjacent queries share one scan and their chunk unions; Sec. 7.1 for the
+ * serving setting). Token t of sequence b gets exactly the decode result of
+ * a query at position cache_len[b]-T+t (its own window, candidates and
+ * top-K). The landmark keys of a (sequence, kv head) are read once for all
+ * T x G scoring queries.
+ *   base              as in hils_decode_args, except the token-major
+ *                     query/output layouts:
+ *     Q, Qs   [B, T, Hq, d]      O [B, T, Hq, d]
+ *     idx     [B, T, Hkv, K]     sel_score [B, T, Hq, K] (nullable)
+ *   T                 tokens per sequence, 1 <= T, T * (Hq/Hkv) <= 32
+ *   block_table       nullable: when given, base.Kc / base.V are the page
+ *                     pool of hils_decode_paged_args and n_pages its size
+ * cache_len[b] must lie in [T, Lmax] (else HILS_ERR_DEVICE_BAD_LENGTH in
+ * the status word). Supported: bf16, d in {64,128}, S in {64,128}, G <= 8;
+ * other shapes return HILS_ERR_UNSUPPORTED. T = 1 is hils_fwd_decode
+ * (or hils_fwd_decode_paged).
+ */
+typedef struct {
+    hils_decode_args base;
+    int32_t T;
+    const int32_t *block_table;     /* device, nullable */
+    int32_t n_pages;
+} hils_decode_multi_args;
+
+hils_status hils_decode_multi_workspace_size(const hils_decode_multi_args *args,
+                                             size_t *bytes);
+hils_status hils_fwd_decode_multi(const hils_decode_multi_args *args, void *stream);
+
+/*
  * Landmark summaries of the chunks: the (k', b') inputs of the scoring step.
  * "Hierarchical Sparse Attention Done Right", Sec. 3 (answering RQ1, the
  * surrogate of Eq. 7): for every full chunk c (nC = floor(N/S) of them) of

@@ -234,3 +234,36 @@ def test_decode_paged_validation(L):
     d.base.dtype = hils.F32               # no f32 paged kernels
     assert L.hils_fwd_decode_paged(ctypes.byref(d), None) == 2
     assert L.hils_fwd_decode_paged(None, None) == 1
+
+
+def _multi(**kw):
+    fake = 1 << 40
+    base = hils.DecodeArgs(hils.BF16, 2, 8, 2, 1024, 128, 64, 128, 8,
+                           None, fake, None, fake, fake, fake, fake, fake,
+                           fake, fake, None, fake, 1 << 30, None)
+    a = dict(base=base, T=4, block_table=None, n_pages=0)
+    a.update(kw)
+    return hils.DecodeMultiArgs(**a)
+
+
+def test_decode_multi_validation(L):
+    """Multi-token records are checked on the host before any launch (only
+    records that fail a check are passed to the compute entry point)."""
+    hm = (ctypes.c_int32 * 8)(*[h // 4 for h in range(8)])
+    a = _multi()
+    a.base.head_map = ctypes.cast(hm, ctypes.c_void_p)
+    n = ctypes.c_size_t(0)
+    rc = L.hils_decode_multi_workspace_size(ctypes.byref(a), ctypes.byref(n))
+    assert rc in (0, 2)                   # 2 without a CUDA driver
+    assert rc == 2 or n.value > 0
+    fake = 1 << 40
+    for kw, code in [(dict(T=0), 1), (dict(T=2000), 1), (dict(T=9), 2),
+                     (dict(block_table=fake, n_pages=0), 1)]:
+        b = _multi(**kw)
+        b.base.head_map = ctypes.cast(hm, ctypes.c_void_p)
+        assert L.hils_fwd_decode_multi(ctypes.byref(b), None) == code, kw
+    d = _multi()
+    d.base.head_map = ctypes.cast(hm, ctypes.c_void_p)
+    d.base.dtype = hils.F32               # no f32 multi-token kernels
+    assert L.hils_fwd_decode_multi(ctypes.byref(d), None) == 2
+    assert L.hils_fwd_decode_multi(None, None) == 1

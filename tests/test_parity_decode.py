@@ -181,3 +181,86 @@ def test_decode_paged_bad_page_reported(cuda_device):
                           sh.K, status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 7          # HILS_ERR_DEVICE_BAD_LENGTH
+
+
+# ---------------------------------------------------------------- multi-token
+def _multi_inputs(name, T, seed, cuda_device):
+    """Decode inputs plus T query tokens per sequence, token-major [B,T,Hq,d].
+    cache_len counts the T new tokens (already in the cache)."""
+    sh, lens = CASES[name]
+    lens = [max(l, T) for l in lens]
+    inp = synth.make_decode(sh, seed=seed, device=cuda_device, cache_len=lens)
+    g = torch.Generator(device="cpu").manual_seed(seed + 17)
+    Qm = torch.randn(sh.B, T, sh.Hq, sh.d, generator=g).to(inp["Q"].dtype)
+    return sh, lens, inp, Qm.to(cuda_device).contiguous()
+
+
+def _token_view(inp, sh, lens, Qm, T, t):
+    """The plain decode record of token t: its query, the cache length that
+    puts it at position cache_len - T + t."""
+    cl = torch.tensor([l - (T - 1 - t) for l in lens], dtype=torch.int32,
+                      device=inp["cache_len"].device)
+    return dict(inp, Q=Qm[:, t].contiguous(), cache_len=cl)
+
+
+def run_multi(inp, sh, Qm, block_table=None, K=None, V=None, status=None):
+    O, idx = hils.fwd_decode_multi(Qm, inp["K"] if K is None else K,
+                                   inp["V"] if V is None else V, inp["Klm"],
+                                   inp["bias"], inp["cache_len"],
+                                   inp["head_map"], sh.S, sh.W, sh.K,
+                                   block_table=block_table, status=status)
+    torch.cuda.synchronize()
+    return O, idx
+
+
+@pytest.mark.parametrize("name,T", [("bf16_ragged", 2), ("bf16_ragged", 4),
+                                    ("bf16_short", 3), ("bf16_d64_S128", 4),
+                                    ("bf16_ragged", 8)])
+def test_decode_multi_matches_oracle_per_token(name, T, cuda_device):
+    """Token t of a T-token step is the decode of a query at position
+    cache_len - T + t: idx bit-exact (up to near ties) and O within the bf16
+    bound against the oracle, and idx equal to the single-token step's."""
+    sh, lens, inp, Qm = _multi_inputs(name, T, 301 + T, cuda_device)
+    O, idx = run_multi(inp, sh, Qm)
+    for t in range(T):
+        sub = _token_view(inp, sh, lens, Qm, T, t)
+        parity.check_decode(sub, O[:, t], idx[:, t])
+        _, idx1 = run_decode(sub)
+        assert torch.equal(idx[:, t], idx1), f"token {t}: idx differs from single-token decode"
+
+
+def test_decode_multi_T1_equals_decode(cuda_device):
+    """T = 1 runs exactly the plain decode step: bit-identical O and idx."""
+    sh, lens, inp, Qm = _multi_inputs("bf16_ragged", 1, 311, cuda_device)
+    O, idx = run_multi(inp, sh, Qm)
+    O1, idx1 = run_decode(dict(inp, Q=Qm[:, 0].contiguous()))
+    assert torch.equal(idx[:, 0], idx1)
+    assert torch.equal(O[:, 0], O1)
+
+
+def test_decode_multi_paged_equals_contiguous(cuda_device):
+    """The multi-token step over a page pool gives bit-identical results."""
+    T = 4
+    sh, lens, inp, Qm = _multi_inputs("bf16_ragged", T, 321, cuda_device)
+    O_ref, idx_ref = run_multi(inp, sh, Qm)
+    Kp, Vp, bt = _to_pages(inp, sh, seed=9)
+    O, idx = run_multi(inp, sh, Qm, block_table=bt, K=Kp, V=Vp)
+    assert torch.equal(idx, idx_ref)
+    assert torch.equal(O, O_ref)
+
+
+def test_decode_multi_short_cache_reported(cuda_device):
+    """cache_len below T is reported in the status word; other sequences are
+    still computed."""
+    T = 4
+    sh, lens, inp, Qm = _multi_inputs("bf16_short", T, 331, cuda_device)
+    inp = dict(inp, cache_len=torch.tensor([lens[0], 2], dtype=torch.int32,
+                                           device=cuda_device))
+    st = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    O, idx = run_multi(inp, sh, Qm, status=st)
+    assert int(st.item()) == 7          # HILS_ERR_DEVICE_BAD_LENGTH
+    sub = _token_view(dict(inp, Q=inp["Q"][:1], K=inp["K"][:1], V=inp["V"][:1],
+                           Klm=inp["Klm"][:1], bias=inp["bias"][:1],
+                           shape=sh.with_(B=1)),
+                      sh, lens[:1], Qm[:1], T, T - 1)
+    parity.check_decode(sub, O[:1, T - 1], idx[:1, T - 1])

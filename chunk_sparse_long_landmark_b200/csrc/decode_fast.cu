@@ -345,9 +345,64 @@ __device__ int block_excl_scan(int v, int *scratch, int *total) {
 }
 
 constexpr int kSelPer = 16;                      // chunks per thread (<= 16384)
+
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
+    const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
+    const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
+    return ((uint64_t)hi << 32) | lo;
+}
+
+// Sorts the warp's 64 values, element e = 2*lane + j in v[j], into
+// descending order (bitonic network: 21 compare-exchange rounds, partners
+// at distance 1 in the same lane, the others one shuffle away).
+__device__ __forceinline__ void warp_sort64_desc(uint64_t v[2]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int k = 2; k <= 64; k <<= 1) {
+#pragma unroll
+        for (int s = k >> 1; s >= 1; s >>= 1) {
+            uint64_t o[2];
+            if (s == 1) {
+                o[0] = v[1];
+                o[1] = v[0];
+            } else {
+                o[0] = shfl_xor_u64(v[0], s >> 1);
+                o[1] = shfl_xor_u64(v[1], s >> 1);
+            }
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int e = 2 * lane + j;
+                // the lower element of a pair keeps the larger value in a
+                // descending block ((e & k) == 0), the smaller otherwise
+                const bool keep_max = ((e & s) == 0) == ((e & k) == 0);
+                v[j] = keep_max ? (v[j] > o[j] ? v[j] : o[j])
+                                : (v[j] < o[j] ? v[j] : o[j]);
+            }
+        }
+    }
+}
 constexpr int kCandCap = 1024;                   // threshold-path candidate list
 constexpr int kMaxSplits = 64;                   // staged landmark-split partials
 
+// s^ of head slot hh for this thread's chunks cbeg .. cbeg+per-1 (16-byte
+// loads; rows are padded to a multiple of 4, values past nc are read but
+// never turned into keys)
+template <int PER>
+__device__ __forceinline__ void sel_load_row(const float *ss, int ncs, int hh,
+                                             int cbeg, int per, int nc,
+                                             float (&v)[PER]) {
+    const float *row = ss + (int64_t)hh * ncs;
+#pragma unroll
+    for (int q4 = 0; q4 < PER / 4; ++q4) {
+        float4 f = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+        if (4 * q4 < per && cbeg + 4 * q4 < nc)
+            f = __ldcg(reinterpret_cast<const float4 *>(row + cbeg + 4 * q4));
+        v[4 * q4 + 0] = f.x; v[4 * q4 + 1] = f.y;
+        v[4 * q4 + 2] = f.z; v[4 * q4 + 3] = f.w;
+    }
+}
+
+template <int PER>
 __global__ void __launch_bounds__(kSelThreads)
 dec_select_kernel(const DecParams p) {
     __shared__ float lse[HILS_MAX_GROUP];
@@ -372,6 +427,15 @@ dec_select_kernel(const DecParams p) {
     const float *ss = p.ws_s + (int64_t)bgt * G * p.ncs;
     grid_dep_wait();                             // dec_score's s^ and partials
     grid_dep_launch();                           // dec_attend may start now
+
+    // chunks of this thread: c = tid * per + q, per a multiple of 4 (16-byte
+    // loads), at most PER. The s^ of the first two heads are loaded before
+    // the log-sum-exp merge so both round trips overlap.
+    const int per = ((nc + kSelThreads - 1) / kSelThreads + 3) & ~3;
+    const int cbeg = threadIdx.x * per;
+    float v0[PER], v1[PER];
+    sel_load_row<PER>(ss, p.ncs, 0, cbeg, per, nc, v0);
+    if (G > 1) sel_load_row<PER>(ss, p.ncs, 1, cbeg, per, nc, v1);
 
     // merge the split partials: all loaded at once into shared memory, then
     // folded in split order by one thread per head
@@ -398,48 +462,42 @@ dec_select_kernel(const DecParams p) {
     }
     __syncthreads();
 
-    // group scores of this thread's contiguous chunks c = tid * per + q
-    // a multiple of 4 (16-byte loads), at most kSelPer
-    const int per = ((nc + kSelThreads - 1) / kSelThreads + 3) & ~3;
-    const int cbeg = threadIdx.x * per;
-    // head by head, the thread's chunks loaded together (one round trip
-    // per head instead of one per chunk and head)
-    float amax[kSelPer];
+    // group scores a_c = max_h (s^_hc - LSE_h), heads two at a time
+    float amax[PER];
 #pragma unroll
-    for (int q = 0; q < kSelPer; ++q) amax[q] = -INFINITY;
-    for (int hh = 0; hh < G; ++hh) {
-        const float *row = ss + (int64_t)hh * p.ncs;
-        const float lh = lse[hh];
-        float v[kSelPer];
+    for (int q = 0; q < PER; ++q) amax[q] = v0[q] - lse[0];
+    if (G > 1) {
 #pragma unroll
-        for (int q4 = 0; q4 < kSelPer / 4; ++q4) {
-            // rows are padded to a multiple of 4: values past nc are read
-            // but never turned into keys
-            float4 f = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-            if (4 * q4 < per && cbeg + 4 * q4 < nc)
-                f = __ldcg(reinterpret_cast<const float4 *>(row + cbeg + 4 * q4));
-            v[4 * q4 + 0] = f.x; v[4 * q4 + 1] = f.y;
-            v[4 * q4 + 2] = f.z; v[4 * q4 + 3] = f.w;
-        }
-#pragma unroll
-        for (int q = 0; q < kSelPer; ++q) amax[q] = fmaxf(amax[q], v[q] - lh);
+        for (int q = 0; q < PER; ++q) amax[q] = fmaxf(amax[q], v1[q] - lse[1]);
     }
-    uint32_t key[kSelPer];
+    for (int hh = 2; hh < G; hh += 2) {
+        sel_load_row<PER>(ss, p.ncs, hh, cbeg, per, nc, v0);
+        if (hh + 1 < G) sel_load_row<PER>(ss, p.ncs, hh + 1, cbeg, per, nc, v1);
+        const float l0 = lse[hh], l1 = hh + 1 < G ? lse[hh + 1] : 0.f;
 #pragma unroll
-    for (int q = 0; q < kSelPer; ++q)                // 0: below every real key
+        for (int q = 0; q < PER; ++q) amax[q] = fmaxf(amax[q], v0[q] - l0);
+        if (hh + 1 < G) {
+#pragma unroll
+            for (int q = 0; q < PER; ++q) amax[q] = fmaxf(amax[q], v1[q] - l1);
+        }
+    }
+    uint32_t key[PER];
+#pragma unroll
+    for (int q = 0; q < PER; ++q)                    // 0: below every real key
         key[q] = (q < per && cbeg + q < nc) ? order_key(amax[q]) : 0u;
     const int nsel = min(nc, K);
 
     // Threshold path. Each warp's two largest keys belong to distinct
     // chunks, so the K-th largest of those 2 x 32 values is a lower bound on
     // the K-th largest key (K <= 64). Only keys at or above it become
-    // candidates; their exact ranks (ties: lower chunk first) are counted
-    // over the short list. A list longer than kCandCap (exact or near ties
-    // over many chunks) falls through to the radix select below.
+    // candidates. Up to 64 candidates are ordered by one warp (sort by key,
+    // ties to the lower chunk, then the first K by chunk); a longer list
+    // gets exact ranks counted over it; one longer than kCandCap (exact or
+    // near ties over many chunks) falls through to the radix select below.
     if (nc > K && K <= 2 * (kSelThreads / 32)) {
         uint32_t t1 = 0u, t2 = 0u;               // this thread's two largest
 #pragma unroll
-        for (int q = 0; q < kSelPer; ++q) {
+        for (int q = 0; q < PER; ++q) {
             const uint32_t k = key[q];
             t2 = max(t2, min(t1, k));
             t1 = max(t1, k);
@@ -456,22 +514,18 @@ dec_select_kernel(const DecParams p) {
         if (threadIdx.x == 0) ncand = 0;
         __syncthreads();
         if (warp == 0) {
-            // largest v among the 64 with at least K of them >= v
-            uint32_t best = 0u;
-#pragma unroll
-            for (int s2 = 0; s2 < 2; ++s2) {
-                const uint32_t v = wtop[2 * lane + s2];
-                int ge = 0;
-                for (int f = 0; f < 2 * (kSelThreads / 32); ++f) ge += (wtop[f] >= v) ? 1 : 0;
-                if (ge >= K) best = max(best, v);
-            }
-            for (int o = 1; o < 32; o <<= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
-            if (lane == 0) sh_tau = best;
+            // the K-th largest of the 64 warp maxima
+            uint64_t w[2] = {(uint64_t)wtop[2 * lane] << 32,
+                             (uint64_t)wtop[2 * lane + 1] << 32};
+            warp_sort64_desc(w);
+            const uint64_t wk = __shfl_sync(0xffffffffu, (uint32_t)(w[(K - 1) & 1] >> 32),
+                                            (K - 1) >> 1);
+            if (lane == 0) sh_tau = (uint32_t)wk;
         }
         __syncthreads();
         const uint32_t tau = sh_tau;
 #pragma unroll
-        for (int q = 0; q < kSelPer; ++q) {
+        for (int q = 0; q < PER; ++q) {
             const int c = cbeg + q;
             if (q < per && c < nc && key[q] >= tau) {
                 const int at = atomicAdd(&ncand, 1);
@@ -480,6 +534,39 @@ dec_select_kernel(const DecParams p) {
         }
         __syncthreads();
         const int m = ncand;
+        if (m <= 64) {
+            if (warp == 0) {
+                // by key descending, ties to the lower chunk: (key, ~chunk)
+                uint64_t w[2];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int e = 2 * lane + j;
+                    w[j] = e < m ? ((uint64_t)cand_k[e] << 32) | (0xffffffffu - (uint32_t)cand_c[e])
+                                 : 0ull;
+                }
+                warp_sort64_desc(w);
+                // the first K, by chunk ascending: (1, ~chunk) descending
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int e = 2 * lane + j;
+                    w[j] = e < K ? ((1ull << 32) | (uint32_t)w[j]) : 0ull;
+                }
+                warp_sort64_desc(w);
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int pos = 2 * lane + j;
+                    if (pos < K) {
+                        const int c = (int)(0xffffffffu - (uint32_t)w[j]);
+                        p.idx[(int64_t)bgv * K + pos] = c;
+                        for (int hh = 0; hh < G; ++hh) {
+                            const int h = p.group_heads[g * G + hh];
+                            p.sel[((int64_t)v * p.Hq + h) * K + pos] = ss[(int64_t)hh * p.ncs + c];
+                        }
+                    }
+                }
+            }
+            return;                              // nc > K: no padding
+        }
         if (m <= kCandCap) {
             bool mine = false;
             uint32_t mk = 0u;
@@ -520,7 +607,7 @@ dec_select_kernel(const DecParams p) {
             for (int x = threadIdx.x; x < 256; x += kSelThreads) hist[x] = 0;
             __syncthreads();
 #pragma unroll
-            for (int q = 0; q < kSelPer; ++q) {
+            for (int q = 0; q < PER; ++q) {
                 const int c = cbeg + q;
                 if (q < per && c < nc && (key[q] & pmask) == prefix)
                     atomicAdd(&hist[(key[q] >> shift) & 255], 1);
@@ -561,14 +648,14 @@ dec_select_kernel(const DecParams p) {
     // (chunk order = thread order, then q); positions in ascending chunk order
     int n_eq = 0;
 #pragma unroll
-    for (int q = 0; q < kSelPer; ++q)
+    for (int q = 0; q < PER; ++q)
         if (q < per && cbeg + q < nc && nc > K && key[q] == thr) ++n_eq;
     int tot;
     int rank_eq = block_excl_scan(n_eq, scan_scr, &tot);
     uint32_t selbits = 0u;
     int n_sel = 0;
 #pragma unroll
-    for (int q = 0; q < kSelPer; ++q) {
+    for (int q = 0; q < PER; ++q) {
         const int c = cbeg + q;
         bool sc = false;
         if (q < per && c < nc) {
@@ -1084,7 +1171,13 @@ cudaError_t launch_dec_select(Problem &p, void *ws, cudaStream_t st) {
         else e = launch_score_t<64, 4>(grid, smem, st, tl, d);
     }
     if (e != cudaSuccess) return e;
-    e = launch_dependent(dec_select_kernel, dim3(p.Hkv, p.B * p.T), dim3(kSelThreads), 0, st, d);
+    // chunks per selection thread: the largest candidate count over 1024
+    // threads, in {4, 8, 16}
+    const int per = ((d.ncs + kSelThreads - 1) / kSelThreads + 3) & ~3;
+    const dim3 sg(p.Hkv, p.B * p.T);
+    if (per <= 4) e = launch_dependent(dec_select_kernel<4>, sg, dim3(kSelThreads), 0, st, d);
+    else if (per <= 8) e = launch_dependent(dec_select_kernel<8>, sg, dim3(kSelThreads), 0, st, d);
+    else e = launch_dependent(dec_select_kernel<16>, sg, dim3(kSelThreads), 0, st, d);
     count_launches(2);
     return e != cudaSuccess ? e : cudaGetLastError();
 }

@@ -148,7 +148,12 @@ def decode_multi_bytes(sh, cache_len, T, idx):
 
 # ------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+    """SM clock and clock-event (throttle) reasons sampled during a region.
+
+    A reader thread polls NVML every 5 ms (read-only queries), so even a
+    region of a few tens of milliseconds gets samples. The device is matched
+    by UUID, which holds whatever CUDA_VISIBLE_DEVICES maps it to. Without
+    NVML it falls back to `nvidia-smi -lms 200` on the same UUID."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,"
          "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
          "clocks_event_reasons.hw_thermal_slowdown,"
@@ -157,16 +162,57 @@ class ClockSampler:
 
     def __init__(self, index):
         self.index = index
-        self.proc = None
-        self.path = None
+        self.rows = []
+        self.proc = self.path = self.thread = None
+        self.stop = None
+
+    def _uuid(self):
+        try:
+            import torch
+            u = str(torch.cuda.get_device_properties(self.index).uuid)
+            return u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            return None
 
     def __enter__(self):
+        import threading
+        uuid = self._uuid()
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = (nv.nvmlDeviceGetHandleByUUID(uuid) if uuid
+                 else nv.nvmlDeviceGetHandleByIndex(self.index))
+            smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                                  None) or nv.nvmlDeviceGetCurrentClocksThrottleReasons
+            bits = {"hw": 0x8, "hwt": 0x40, "swt": 0x20, "pcap": 0x4}
+            self.stop = threading.Event()
+
+            def run():
+                while not self.stop.is_set():
+                    try:
+                        r = int(get_reasons(h))
+                        row = dict(sm=float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                   smax=smax,
+                                   power=nv.nvmlDeviceGetPowerUsage(h) / 1e3)
+                        for k, bit in bits.items():
+                            row[k] = "Active" if r & bit else "Not Active"
+                        self.rows.append(row)
+                    except Exception:
+                        pass
+                    self.stop.wait(0.005)
+
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            return self
+        except Exception:
+            self.thread = None
         import tempfile
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                ["nvidia-smi", f"--id={uuid or self.index}", f"--query-gpu={self.Q}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
@@ -174,6 +220,9 @@ class ClockSampler:
         return self
 
     def __exit__(self, *exc):
+        if self.thread is not None:
+            self.stop.set()
+            self.thread.join(timeout=5)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -182,20 +231,19 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        if not self.path or not os.path.exists(self.path):
-            return None
-        rows = []
-        for line in open(self.path):
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                rows.append(dict(sm=float(f[1]), smax=float(f[2]),
-                                 power=float(f[3]), hw=f[5], hwt=f[6],
-                                 swt=f[7], pcap=f[8]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
+        rows = list(self.rows)
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(f[1]), smax=float(f[2]),
+                                     power=float(f[3]), hw=f[5], hwt=f[6],
+                                     swt=f[7], pcap=f[8]))
+                except ValueError:
+                    continue
+            os.unlink(self.path)
         if not rows:
             return None
         reasons = set()
@@ -207,7 +255,8 @@ class ClockSampler:
                     reasons.add(n)
         return {"sm_mhz": statistics.median(r["sm"] for r in rows),
                 "sm_max_mhz": max(r["smax"] for r in rows),
-                "samples": len(rows), "reasons": sorted(reasons)}
+                "samples": len(rows), "reasons": sorted(reasons),
+                "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
 def measured_peaks():

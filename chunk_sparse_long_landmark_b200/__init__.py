@@ -20,7 +20,7 @@ __all__ = [
     "decode_workspace_size", "PrefillArgs", "DecodeArgs", "STATUS",
     "launch_count", "fwd_decode_noalloc", "build_landmarks", "LandmarkArgs",
     "chunk_overlap", "fwd_decode_paged", "DecodePagedArgs",
-    "fwd_decode_multi", "DecodeMultiArgs",
+    "fwd_decode_multi", "DecodeMultiArgs", "bwd_prefill", "BackwardArgs",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -43,6 +43,7 @@ symbols = [
     "hils_build_landmarks", "hils_chunk_overlap",
     "hils_decode_paged_workspace_size", "hils_fwd_decode_paged",
     "hils_decode_multi_workspace_size", "hils_fwd_decode_multi",
+    "hils_bwd_prefill_workspace_size", "hils_bwd_prefill",
 ]
 
 
@@ -76,6 +77,16 @@ class DecodeArgs(ctypes.Structure):
 
 class DecodePagedArgs(ctypes.Structure):
     _fields_ = [("base", DecodeArgs), ("block_table", _p), ("n_pages", _i)]
+
+
+class BackwardArgs(ctypes.Structure):
+    _fields_ = [("dtype", _i), ("B", _i), ("Hq", _i), ("Hkv", _i), ("N", _i),
+                ("d", _i), ("S", _i), ("W", _i), ("K", _i), ("head_map", _p),
+                ("Q", _p), ("Qs", _p), ("Kc", _p), ("V", _p), ("Klm", _p),
+                ("bias", _p), ("dO", _p), ("idx", _p), ("dQ", _p),
+                ("dQs", _p), ("dK", _p), ("dV", _p), ("dKlm", _p),
+                ("dbias", _p), ("workspace", _p),
+                ("workspace_bytes", ctypes.c_size_t)]
 
 
 class DecodeMultiArgs(ctypes.Structure):
@@ -134,6 +145,12 @@ def lib():
             L.hils_fwd_decode_multi.restype = ctypes.c_int
             L.hils_fwd_decode_multi.argtypes = [ctypes.POINTER(DecodeMultiArgs),
                                                 ctypes.c_void_p]
+            L.hils_bwd_prefill_workspace_size.restype = ctypes.c_int
+            L.hils_bwd_prefill_workspace_size.argtypes = [
+                ctypes.POINTER(BackwardArgs), ctypes.POINTER(ctypes.c_size_t)]
+            L.hils_bwd_prefill.restype = ctypes.c_int
+            L.hils_bwd_prefill.argtypes = [ctypes.POINTER(BackwardArgs),
+                                           ctypes.c_void_p]
             L.hils_chunk_overlap.restype = ctypes.c_int
             L.hils_chunk_overlap.argtypes = [_p] + [_i] * 6 + [_p] * 4
             _lib = L
@@ -474,3 +491,51 @@ def fwd_decode_multi(Q, Kc, V, Klm, bias, cache_len, head_map, S, W, topk,
     if rc:
         raise HilsError(rc, "hils_fwd_decode_multi")
     return out, idx
+
+
+def bwd_prefill(Q, K, V, Klm, bias, head_map, S, W, idx, dO, Qs=None,
+                grads=None, workspace=None, stream=None):
+    """Backward of the prefill forward for a fixed selection, through
+    hils_bwd_prefill. Returns a dict of float32 gradients dQ, dQs (None
+    without Qs: folded into dQ), dK, dV, dKlm, dbias.
+
+    Q/Qs/dO [B,Hq,N,d], K/V [B,Hkv,N,d], Klm [B,Hkv,N//S,d], bias
+    [B,Hkv,N//S] (f32), idx [B,Hkv,N,topk] int32: the forward's selection.
+    `grads` may hold preallocated outputs under the same keys."""
+    import torch
+    _dev(Q, K, V, Klm, bias, idx, dO, Qs, workspace)
+    B, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    topk = idx.shape[-1]
+    hm = _head_map_array(head_map, Hq)
+    f32 = dict(dtype=torch.float32, device=Q.device)
+    g = dict(grads or {})
+    g.setdefault("dQ", torch.empty(B, Hq, N, d, **f32))
+    g.setdefault("dQs", torch.empty(B, Hq, N, d, **f32) if Qs is not None else None)
+    g.setdefault("dK", torch.empty(B, Hkv, N, d, **f32))
+    g.setdefault("dV", torch.empty(B, Hkv, N, d, **f32))
+    g.setdefault("dKlm", torch.empty(B, Hkv, max(N // S, 1), d, **f32))
+    g.setdefault("dbias", torch.empty(B, Hkv, max(N // S, 1), **f32))
+
+    def record(ws):
+        return BackwardArgs(_dtype_code(Q), B, Hq, Hkv, N, d, S, W, topk,
+                            ctypes.cast(hm, ctypes.c_void_p), _ptr(Q),
+                            _ptr(Qs), _ptr(K), _ptr(V), _ptr(Klm), _ptr(bias),
+                            _ptr(dO), _ptr(idx), _ptr(g["dQ"]), _ptr(g["dQs"]),
+                            _ptr(g["dK"]), _ptr(g["dV"]), _ptr(g["dKlm"]),
+                            _ptr(g["dbias"]), _ptr(ws),
+                            0 if ws is None else ws.numel() * ws.element_size())
+
+    if workspace is None:
+        n = ctypes.c_size_t(0)
+        rc = lib().hils_bwd_prefill_workspace_size(ctypes.byref(record(None)),
+                                                   ctypes.byref(n))
+        if rc:
+            raise HilsError(rc, "hils_bwd_prefill_workspace_size")
+        workspace = torch.empty(max(n.value, 1), dtype=torch.uint8,
+                                device=Q.device)
+    rc = lib().hils_bwd_prefill(ctypes.byref(record(workspace)),
+                                _stream_handle(stream))
+    if rc:
+        raise HilsError(rc, "hils_bwd_prefill")
+    return g

@@ -1,0 +1,653 @@
+// backward.cu -- gradients of the HiLS prefill output, selection held fixed.
+//
+// "Hierarchical Sparse Attention Done Right", Sec. 3 (RQ2: the chunk-level
+// softmax fused with the intra-chunk softmax is what lets the language-model
+// loss reach the landmark scores) and Sec. 4 (native sparse training). The
+// top-K choice is discrete; every continuous quantity of the fused output
+// gets its gradient. For one row i, head h (kv group g):
+//   s_j = q.k_j/sqrt(d); sh_c = qs.k'_c/sqrt(d) + b'_c; lz_c = log sum_c e^s
+//   e_j = s_j - lz_c + sh_c (selected chunks), s_j (window); p = softmax(e)
+//   u_j = dO.v_j; D = sum p_j u_j; L = log(sum_c e^{sh_c} + sum_win e^{s_j})
+//   chunk c: P_c = e^{sh_c - L}, Ubar_c = sum_{j in c} e^{s_j - lz_c} u_j,
+//            ds_j = p_j (u_j - Ubar_c), dsh_c = P_c (Ubar_c - D)
+//   window:  p_j = e^{s_j - L}, ds_j = p_j (u_j - D)
+//   dV_j += p_j dO; dK_j += ds_j q/sqrt(d); dq += ds_j k_j/sqrt(d)
+//   dqs += dsh_c k'_c/sqrt(d); dk'_c += dsh_c qs/sqrt(d); db'_c += dsh_c
+//
+// Two kernels, no floating-point atomics (every output element is summed by
+// one thread in a fixed order, so results are bitwise reproducible):
+//   bwd_rows  one warp per (b, g, i) with the group's G heads: two passes
+//             over the row's tokens (lane per token) give lz_c, L, D, then
+//             p and ds; dq accumulates with lane l owning d/32 dims. Writes
+//             dQ (dQs) and per (row, head) L, D and per (row, head, chunk)
+//             lz, P, Ubar for the key-side kernel.
+//   bwd_keys  one CTA per (b, g, chunk of S tokens): the query rows that
+//             selected the chunk (found by scanning idx, ascending) and the
+//             rows whose window covers it, in ascending order; thread
+//             (token, quarter of dims) keeps its K/V slice and its dK/dV
+//             accumulators in registers. Also dk'_c and db'_c.
+// Inputs f32 or bf16, arithmetic and outputs f32.
+#include <math.h>
+#include <stdint.h>
+
+#include "hils_fast.cuh"
+
+namespace hils {
+namespace {
+
+__device__ __forceinline__ float ld_f(const float *p) { return *p; }
+__device__ __forceinline__ float ld_f(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+struct BwdParams {
+    const void *Q, *Qs, *Kc, *Vc, *Klm, *dO;
+    const float *bias;
+    const int32_t *idx;
+    float *dQ, *dQs, *dK, *dV, *dKlm, *dbias;
+    float *rowstat;     // [B, Hq, N, 2]: L, D
+    float *chunkstat;   // [B, Hq, N, K, 3]: lz, P, Ubar (valid selected entries)
+    int B, Hq, Hkv, G, N, S, W, K, nC;
+    float inv_sqrt_d;
+    int16_t group_heads[kMaxHeads];
+};
+
+__device__ __forceinline__ void bwd_bounds(int64_t i, int S, int W, int64_t *w0,
+                                           int64_t *nc) {
+    window_bounds(i, S, W, w0, nc);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+
+constexpr int kRowWarps = 4;
+
+// Shared memory of one warp in bwd_rows: the G heads' q, qs and dO rows
+// (f32), the row's valid selected chunks with their idx position, s^, lz and
+// Ubar.
+template <int D, int GM>
+struct RowSmem {
+    float q[GM][D], qs[GM][D], go[GM][D];
+    int chunk[HILS_MAX_TOPK], kpos[HILS_MAX_TOPK];
+    float sh[GM][HILS_MAX_TOPK], lz[GM][HILS_MAX_TOPK], ub[GM][HILS_MAX_TOPK];
+};
+
+// s = q_h . k_j and u = dO_h . v_j for the G heads, one token per lane.
+template <typename T, int D, int GM>
+__device__ __forceinline__ void token_dots(const RowSmem<D, GM> &sm, int G,
+                                           const T *krow, const T *vrow,
+                                           float *s, float *u) {
+#pragma unroll
+    for (int h = 0; h < GM; ++h) s[h] = u[h] = 0.f;
+#pragma unroll 4
+    for (int k = 0; k < D; ++k) {
+        const float kv = ld_f(krow + k), vv = ld_f(vrow + k);
+#pragma unroll
+        for (int h = 0; h < GM; ++h)
+            if (h < G) {
+                s[h] = fmaf(sm.q[h][k], kv, s[h]);
+                u[h] = fmaf(sm.go[h][k], vv, u[h]);
+            }
+    }
+}
+
+template <typename T, int D, int GM>
+__global__ void __launch_bounds__(kRowWarps * 32)
+bwd_rows_kernel(const BwdParams p) {
+    constexpr int DL = D / 32;                   // dims per lane
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    RowSmem<D, GM> &sm = reinterpret_cast<RowSmem<D, GM> *>(smem_raw)[warp];
+    const int64_t row = (int64_t)blockIdx.x * kRowWarps + warp;     // (b, g, i)
+    if (row >= (int64_t)p.B * p.Hkv * p.N) return;
+    const int i = (int)(row % p.N);
+    const int g = (int)((row / p.N) % p.Hkv);
+    const int b = (int)(row / ((int64_t)p.N * p.Hkv));
+    const int G = p.G;
+    const float isd = p.inv_sqrt_d;
+    const T *Kg = reinterpret_cast<const T *>(p.Kc) + ((int64_t)b * p.Hkv + g) * p.N * D;
+    const T *Vg = reinterpret_cast<const T *>(p.Vc) + ((int64_t)b * p.Hkv + g) * p.N * D;
+    const T *Lg = reinterpret_cast<const T *>(p.Klm) + ((int64_t)b * p.Hkv + g) * p.nC * D;
+    const T *Qs = reinterpret_cast<const T *>(p.Qs ? p.Qs : p.Q);
+
+    // the G heads' rows -> shared memory (f32)
+    for (int h = 0; h < G; ++h) {
+        const int hq = p.group_heads[g * G + h];
+        const int64_t off = (((int64_t)b * p.Hq + hq) * p.N + i) * D;
+        for (int k = lane; k < D; k += 32) {
+            sm.q[h][k] = ld_f(reinterpret_cast<const T *>(p.Q) + off + k);
+            sm.qs[h][k] = ld_f(Qs + off + k);
+            sm.go[h][k] = ld_f(reinterpret_cast<const T *>(p.dO) + off + k);
+        }
+    }
+    int64_t w0, nc;
+    bwd_bounds(i, p.S, p.W, &w0, &nc);
+    // valid selected chunks (ascending, entries outside C_i ignored)
+    const int32_t *ir = p.idx + (((int64_t)b * p.Hkv + g) * p.N + i) * p.K;
+    int nsel = 0;
+    for (int k = 0; k < p.K; ++k) {              // uniform over the warp
+        const int c = ir[k];
+        if (c >= 0 && c < nc) {
+            if (lane == 0) { sm.chunk[nsel] = c; sm.kpos[nsel] = k; }
+            ++nsel;
+        }
+    }
+    __syncwarp();
+    // s^ of the selected chunks (warp dot products)
+    for (int n = 0; n < nsel; ++n) {
+        const T *kl = Lg + (int64_t)sm.chunk[n] * D;
+        const float bn = p.bias[((int64_t)b * p.Hkv + g) * p.nC + sm.chunk[n]];
+        for (int h = 0; h < G; ++h) {
+            float a = 0.f;
+#pragma unroll
+            for (int r = 0; r < DL; ++r) a = fmaf(sm.qs[h][lane * DL + r], ld_f(kl + lane * DL + r), a);
+            a = warp_sum(a);
+            if (lane == 0) sm.sh[h][n] = a * isd + bn;
+        }
+    }
+    __syncwarp();
+
+    // ---- pass 1: lz_c and Ubar_c per chunk; window sums; then L and D
+    float s[GM], u[GM];
+    for (int n = 0; n < nsel; ++n) {
+        const int64_t j0 = (int64_t)sm.chunk[n] * p.S;
+        float m[GM], z[GM], zu[GM];
+#pragma unroll
+        for (int h = 0; h < GM; ++h) { m[h] = -INFINITY; z[h] = zu[h] = 0.f; }
+        for (int t = lane; t < p.S; t += 32) {   // online per lane
+            token_dots<T, D, GM>(sm, G, Kg + (j0 + t) * D, Vg + (j0 + t) * D, s, u);
+#pragma unroll
+            for (int h = 0; h < GM; ++h) {
+                const float x = s[h] * isd;
+                const float mn = fmaxf(m[h], x);
+                const float f = expf(m[h] - mn), e = expf(x - mn);
+                z[h] = z[h] * f + e;
+                zu[h] = zu[h] * f + e * u[h];
+                m[h] = mn;
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < GM; ++h) {
+            if (h >= G) break;
+            const float M = warp_max(m[h]);
+            const float f = (m[h] == -INFINITY) ? 0.f : expf(m[h] - M);
+            const float Z = warp_sum(z[h] * f), ZU = warp_sum(zu[h] * f);
+            if (lane == 0) {
+                sm.lz[h][n] = M + logf(Z);
+                sm.ub[h][n] = ZU / Z;
+            }
+        }
+    }
+    const int64_t nw = (int64_t)i - w0 + 1;      // window tokens
+    float wm[GM], wz[GM], wzu[GM];
+#pragma unroll
+    for (int h = 0; h < GM; ++h) { wm[h] = -INFINITY; wz[h] = wzu[h] = 0.f; }
+    for (int64_t t = lane; t < nw; t += 32) {
+        const int64_t j = w0 + t;
+        token_dots<T, D, GM>(sm, G, Kg + j * D, Vg + j * D, s, u);
+#pragma unroll
+        for (int h = 0; h < GM; ++h) {
+            const float x = s[h] * isd;
+            const float mn = fmaxf(wm[h], x);
+            const float f = expf(wm[h] - mn), e = expf(x - mn);
+            wz[h] = wz[h] * f + e;
+            wzu[h] = wzu[h] * f + e * u[h];
+            wm[h] = mn;
+        }
+    }
+    __syncwarp();
+    float Lr[GM], Dr[GM];
+#pragma unroll
+    for (int h = 0; h < GM; ++h) {
+        Lr[h] = Dr[h] = 0.f;
+        if (h >= G) continue;
+        const float M = warp_max(wm[h]);
+        const float f = (wm[h] == -INFINITY) ? 0.f : expf(wm[h] - M);
+        const float Zw = warp_sum(wz[h] * f), ZUw = warp_sum(wzu[h] * f);
+        float top = M;                           // window holds token i: M finite
+        for (int n = 0; n < nsel; ++n) top = fmaxf(top, sm.sh[h][n]);
+        float tot = Zw * expf(M - top);
+        for (int n = 0; n < nsel; ++n) tot += expf(sm.sh[h][n] - top);
+        const float L = top + logf(tot);
+        float Dv = ZUw * expf(M - L);
+        for (int n = 0; n < nsel; ++n) Dv += expf(sm.sh[h][n] - L) * sm.ub[h][n];
+        Lr[h] = L;
+        Dr[h] = Dv;
+    }
+
+    // ---- pass 2: p, ds; dq with lane l owning dims l*DL .. l*DL+DL-1
+    float dq[GM][DL], dqs[GM][DL];
+#pragma unroll
+    for (int h = 0; h < GM; ++h)
+#pragma unroll
+        for (int r = 0; r < DL; ++r) dq[h][r] = dqs[h][r] = 0.f;
+    // contributions of tokens j0 + t (t < cnt, lane = token) with ds[h]
+    auto accumulate = [&](int64_t j0, int cnt, const float *ds) {
+        for (int tt = 0; tt < cnt; ++tt) {
+            const T *kr = Kg + (j0 + tt) * D + lane * DL;
+            float kv[DL];
+#pragma unroll
+            for (int r = 0; r < DL; ++r) kv[r] = ld_f(kr + r);
+#pragma unroll
+            for (int h = 0; h < GM; ++h) {
+                if (h >= G) break;
+                const float dsv = __shfl_sync(0xffffffffu, ds[h], tt);
+#pragma unroll
+                for (int r = 0; r < DL; ++r) dq[h][r] = fmaf(dsv, kv[r], dq[h][r]);
+            }
+        }
+    };
+    float ds[GM];
+    for (int n = 0; n < nsel; ++n) {
+        const int64_t j0 = (int64_t)sm.chunk[n] * p.S;
+        for (int t0 = 0; t0 < p.S; t0 += 32) {
+            const int t = t0 + lane;
+            const int cnt = min(32, p.S - t0);
+#pragma unroll
+            for (int h = 0; h < GM; ++h) ds[h] = 0.f;
+            if (t < p.S) {
+                token_dots<T, D, GM>(sm, G, Kg + (j0 + t) * D, Vg + (j0 + t) * D, s, u);
+#pragma unroll
+                for (int h = 0; h < GM; ++h) {
+                    if (h >= G) break;
+                    const float P = expf(sm.sh[h][n] - Lr[h]);
+                    const float pj = P * expf(s[h] * isd - sm.lz[h][n]);
+                    ds[h] = pj * (u[h] - sm.ub[h][n]);
+                }
+            }
+            accumulate(j0 + t0, cnt, ds);
+        }
+        // s^ gradient: dsh = P (Ubar - D) -> dqs += dsh k'_c
+        const T *kl = Lg + (int64_t)sm.chunk[n] * D + lane * DL;
+#pragma unroll
+        for (int h = 0; h < GM; ++h) {
+            if (h >= G) break;
+            const float P = expf(sm.sh[h][n] - Lr[h]);
+            const float dsh = P * (sm.ub[h][n] - Dr[h]);
+#pragma unroll
+            for (int r = 0; r < DL; ++r) dqs[h][r] = fmaf(dsh, ld_f(kl + r), dqs[h][r]);
+        }
+    }
+    for (int64_t t0 = 0; t0 < nw; t0 += 32) {
+        const int64_t t = t0 + lane;
+        const int cnt = (int)min((int64_t)32, nw - t0);
+#pragma unroll
+        for (int h = 0; h < GM; ++h) ds[h] = 0.f;
+        if (t < nw) {
+            const int64_t j = w0 + t;
+            token_dots<T, D, GM>(sm, G, Kg + j * D, Vg + j * D, s, u);
+#pragma unroll
+            for (int h = 0; h < GM; ++h) {
+                if (h >= G) break;
+                const float pj = expf(s[h] * isd - Lr[h]);
+                ds[h] = pj * (u[h] - Dr[h]);
+            }
+        }
+        accumulate(w0 + t0, cnt, ds);
+    }
+
+    // ---- outputs
+    for (int h = 0; h < G; ++h) {
+        const int hq = p.group_heads[g * G + h];
+        const int64_t rq = ((int64_t)b * p.Hq + hq) * p.N + i;
+        float *dq_out = p.dQ + rq * D + lane * DL;
+#pragma unroll
+        for (int r = 0; r < DL; ++r) {
+            float v = dq[h][r] * isd;
+            if (!p.dQs) v += dqs[h][r] * isd;
+            dq_out[r] = v;
+        }
+        if (p.dQs) {
+            float *o = p.dQs + rq * D + lane * DL;
+#pragma unroll
+            for (int r = 0; r < DL; ++r) o[r] = dqs[h][r] * isd;
+        }
+        if (lane == 0) {
+            p.rowstat[rq * 2] = Lr[h];
+            p.rowstat[rq * 2 + 1] = Dr[h];
+        }
+        for (int n = lane; n < nsel; n += 32) {
+            float *cs = p.chunkstat + (rq * p.K + sm.kpos[n]) * 3;
+            cs[0] = sm.lz[h][n];
+            cs[1] = expf(sm.sh[h][n] - Lr[h]);
+            cs[2] = sm.ub[h][n];
+        }
+    }
+}
+
+// ------------------------------------------------------------------ keys
+constexpr int kKeyBatch = 8;                     // (row, head) pairs per round
+
+template <int D, int GM>
+struct KeySmem {
+    float q[kKeyBatch][D], go[kKeyBatch][D], qs[kKeyBatch][D];
+    // per pair: chunk role (lz, P, Ubar), window role (L, D, -); the row's
+    // token range inside the chunk; dsh = P (Ubar - D) (chunk role)
+    float a0[kKeyBatch], a1[kKeyBatch], a2[kKeyBatch], dsh[kKeyBatch];
+    int lo[kKeyBatch], hi[kKeyBatch];
+    float dklm[D];
+    float dbias;
+    int list_i[1024], list_k[1024];              // rows of this round
+    int nlist;
+    int scan[33];
+};
+
+template <typename T, int D, int S_TOK, int GM>
+__global__ void __launch_bounds__(S_TOK * 4)
+bwd_keys_kernel(const BwdParams p) {
+    constexpr int DQ = D / 4;                    // dims per thread
+    constexpr int NT = S_TOK * 4;
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    KeySmem<D, GM> &sm = *reinterpret_cast<KeySmem<D, GM> *>(smem_raw);
+    const int nchunks = (p.N + S_TOK - 1) / S_TOK;
+    const int c = blockIdx.x % nchunks;
+    const int g = (blockIdx.x / nchunks) % p.Hkv;
+    const int b = blockIdx.x / (nchunks * p.Hkv);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int jl = tid >> 2, qd = tid & 3;
+    const int64_t j = (int64_t)c * S_TOK + jl;   // this thread's token
+    const bool jok = j < p.N;
+    const int G = p.G;
+    const float isd = p.inv_sqrt_d;
+    const int64_t bg = (int64_t)b * p.Hkv + g;
+    float kreg[DQ], vreg[DQ], adk[DQ], adv[DQ];
+    {
+        const T *kr = reinterpret_cast<const T *>(p.Kc) + (bg * p.N + (jok ? j : 0)) * D + qd * DQ;
+        const T *vr = reinterpret_cast<const T *>(p.Vc) + (bg * p.N + (jok ? j : 0)) * D + qd * DQ;
+#pragma unroll
+        for (int r = 0; r < DQ; ++r) {
+            kreg[r] = jok ? ld_f(kr + r) : 0.f;
+            vreg[r] = jok ? ld_f(vr + r) : 0.f;
+            adk[r] = adv[r] = 0.f;
+        }
+    }
+    for (int k = tid; k < D; k += NT) sm.dklm[k] = 0.f;
+    if (tid == 0) sm.dbias = 0.f;
+    const T *Qp = reinterpret_cast<const T *>(p.Q);
+    const T *Qsp = reinterpret_cast<const T *>(p.Qs ? p.Qs : p.Q);
+    const T *dOp = reinterpret_cast<const T *>(p.dO);
+    const bool is_lm = c < p.nC;                 // a complete chunk: selectable
+
+    // process the (row, head) pairs of rows list_i[0..nlist) in batches
+    auto run_rows = [&](int role) {
+        const int npairs = sm.nlist * G;
+        for (int e0 = 0; e0 < npairs; e0 += kKeyBatch) {
+            const int ne = min(kKeyBatch, npairs - e0);
+            __syncthreads();                     // previous batch consumed
+            for (int e = warp; e < ne; e += NT / 32) {
+                const int pr = e0 + e;
+                const int ri = sm.list_i[pr / G], h = pr % G;
+                const int hq = p.group_heads[g * G + h];
+                const int64_t rq = ((int64_t)b * p.Hq + hq) * p.N + ri;
+                for (int k = lane; k < D; k += 32) {
+                    sm.q[e][k] = ld_f(Qp + rq * D + k);
+                    sm.go[e][k] = ld_f(dOp + rq * D + k);
+                    if (role == 0) sm.qs[e][k] = ld_f(Qsp + rq * D + k);
+                }
+                if (lane == 0) {
+                    if (role == 0) {             // lz, P, Ubar and D of the row
+                        const float *cs = p.chunkstat + (rq * p.K + sm.list_k[pr / G]) * 3;
+                        sm.a0[e] = cs[0];
+                        sm.a1[e] = cs[1];
+                        sm.a2[e] = cs[2];
+                        sm.dsh[e] = cs[1] * (cs[2] - p.rowstat[rq * 2 + 1]);
+                        sm.lo[e] = 0;
+                        sm.hi[e] = S_TOK - 1;
+                    } else {                     // L, D and the window's span
+                        sm.a0[e] = p.rowstat[rq * 2];
+                        sm.a1[e] = p.rowstat[rq * 2 + 1];
+                        int64_t w0, nc;
+                        bwd_bounds(ri, p.S, p.W, &w0, &nc);
+                        const int64_t base = (int64_t)c * S_TOK;
+                        sm.lo[e] = (int)max((int64_t)0, w0 - base);
+                        sm.hi[e] = (int)min((int64_t)S_TOK - 1, (int64_t)ri - base);
+                    }
+                }
+            }
+            __syncthreads();
+            for (int e = 0; e < ne; ++e) {       // fixed order: deterministic
+                float sp = 0.f, up = 0.f;
+#pragma unroll
+                for (int r = 0; r < DQ; ++r) {
+                    sp = fmaf(sm.q[e][qd * DQ + r], kreg[r], sp);
+                    up = fmaf(sm.go[e][qd * DQ + r], vreg[r], up);
+                }
+                sp += __shfl_xor_sync(0xffffffffu, sp, 1);
+                up += __shfl_xor_sync(0xffffffffu, up, 1);
+                sp += __shfl_xor_sync(0xffffffffu, sp, 2);
+                up += __shfl_xor_sync(0xffffffffu, up, 2);
+                const float x = sp * isd;
+                float pj = 0.f, dsj = 0.f;
+                if (jok && jl >= sm.lo[e] && jl <= sm.hi[e]) {
+                    if (role == 0) {
+                        pj = sm.a1[e] * expf(x - sm.a0[e]);
+                        dsj = pj * (up - sm.a2[e]);
+                    } else {
+                        pj = expf(x - sm.a0[e]);
+                        dsj = pj * (up - sm.a1[e]);
+                    }
+                }
+#pragma unroll
+                for (int r = 0; r < DQ; ++r) {
+                    adv[r] = fmaf(pj, sm.go[e][qd * DQ + r], adv[r]);
+                    adk[r] = fmaf(dsj, sm.q[e][qd * DQ + r], adk[r]);
+                }
+            }
+            if (role == 0) {                     // k' and b' of the chunk
+                for (int k = tid; k < D; k += NT) {
+                    float a = sm.dklm[k];
+                    for (int e = 0; e < ne; ++e) a = fmaf(sm.dsh[e], sm.qs[e][k], a);
+                    sm.dklm[k] = a;
+                }
+                if (tid == NT - 1) {
+                    float a = sm.dbias;
+                    for (int e = 0; e < ne; ++e) a += sm.dsh[e];
+                    sm.dbias = a;
+                }
+            }
+        }
+        __syncthreads();
+    };
+
+    // rows that selected chunk c: i >= (c+1) S + W - 1, scanned in rounds of
+    // NT rows; each round's hits are compacted in ascending order
+    if (is_lm) {
+        const int64_t i_min = (int64_t)(c + 1) * p.S + p.W - 1;
+        for (int64_t r0 = i_min; r0 < p.N; r0 += NT) {
+            const int64_t ri = r0 + tid;
+            int hitk = -1;
+            if (ri < p.N) {
+                const int32_t *ir = p.idx + (bg * p.N + ri) * p.K;
+                for (int k = 0; k < p.K; ++k) {
+                    const int v = ir[k];
+                    if (v < 0 || v > c) break;
+                    if (v == c) { hitk = k; break; }
+                }
+            }
+            const unsigned m = __ballot_sync(0xffffffffu, hitk >= 0);
+            __syncthreads();
+            if (lane == 0) sm.scan[warp] = __popc(m);
+            __syncthreads();
+            if (tid == 0) {
+                int acc = 0;
+                for (int w = 0; w < NT / 32; ++w) { const int v = sm.scan[w]; sm.scan[w] = acc; acc += v; }
+                sm.nlist = acc;
+            }
+            __syncthreads();
+            if (hitk >= 0) {
+                const int pos = sm.scan[warp] + __popc(m & ((1u << lane) - 1u));
+                sm.list_i[pos] = (int)ri;
+                sm.list_k[pos] = hitk;
+            }
+            __syncthreads();
+            if (sm.nlist > 0) run_rows(0);
+        }
+    }
+    // rows whose window covers part of the chunk: i in [cS, ...] with w0 <= cS + S - 1
+    {
+        const int64_t base = (int64_t)c * S_TOK;
+        for (int64_t r0 = base; r0 < p.N; r0 += 1024) {
+            __syncthreads();
+            if (tid == 0) {
+                int n = 0;
+                for (int64_t ri = r0; ri < min((int64_t)p.N, r0 + 1024); ++ri) {
+                    int64_t w0, nc;
+                    bwd_bounds(ri, p.S, p.W, &w0, &nc);
+                    if (w0 > base + S_TOK - 1) break;
+                    sm.list_i[n] = (int)ri;
+                    sm.list_k[n] = 0;
+                    ++n;
+                }
+                sm.nlist = n;
+            }
+            __syncthreads();
+            const int n = sm.nlist;
+            if (n > 0) run_rows(1);
+            if (n < 1024) break;
+        }
+    }
+
+    if (jok) {
+        float *dk = p.dK + (bg * p.N + j) * D + qd * DQ;
+        float *dv = p.dV + (bg * p.N + j) * D + qd * DQ;
+#pragma unroll
+        for (int r = 0; r < DQ; ++r) {
+            dk[r] = adk[r] * isd;
+            dv[r] = adv[r];
+        }
+    }
+    __syncthreads();
+    if (is_lm) {
+        for (int k = tid; k < D; k += NT) p.dKlm[(bg * p.nC + c) * D + k] = sm.dklm[k] * isd;
+        if (tid == 0) p.dbias[bg * p.nC + c] = sm.dbias;
+    }
+}
+
+template <typename T, int D, int GM>
+cudaError_t launch_rows_t(const BwdParams &p, cudaStream_t st) {
+    const size_t smem = sizeof(RowSmem<D, GM>) * kRowWarps;
+    cudaError_t e = cudaFuncSetAttribute(bwd_rows_kernel<T, D, GM>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t rows = (int64_t)p.B * p.Hkv * p.N;
+    bwd_rows_kernel<T, D, GM><<<(unsigned)((rows + kRowWarps - 1) / kRowWarps),
+                                kRowWarps * 32, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename T, int D, int GM>
+cudaError_t launch_keys_t(const BwdParams &p, cudaStream_t st) {
+    constexpr int S_TOK = 64;
+    const size_t smem = sizeof(KeySmem<D, GM>);
+    cudaError_t e = cudaFuncSetAttribute(bwd_keys_kernel<T, D, S_TOK, GM>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = (int64_t)p.B * p.Hkv * ((p.N + S_TOK - 1) / S_TOK);
+    bwd_keys_kernel<T, D, S_TOK, GM><<<(unsigned)grid, S_TOK * 4, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename T, int D, int GM>
+cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st) {
+    cudaError_t e = launch_rows_t<T, D, GM>(p, st);
+    if (e != cudaSuccess) return e;
+    return launch_keys_t<T, D, GM>(p, st);
+}
+
+template <typename T, int D>
+cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t st) {
+    if (p.G == 1) return launch_bwd_t<T, D, 1>(p, st);
+    if (p.G == 2) return launch_bwd_t<T, D, 2>(p, st);
+    if (p.G <= 4) return launch_bwd_t<T, D, 4>(p, st);
+    return launch_bwd_t<T, D, 8>(p, st);
+}
+
+bool al16b(const void *q) { return ((uintptr_t)q & 15u) == 0; }
+
+// Shape checks of a backward record; fills p (pointers only when need_ptrs).
+hils_status bwd_problem(const hils_backward_args *a, BwdParams *p, bool need_ptrs,
+                        size_t *ws_bytes) {
+    if (!a) return HILS_ERR_INVALID_ARG;
+    if (a->dtype != HILS_F32 && a->dtype != HILS_BF16) return HILS_ERR_INVALID_ARG;
+    if (a->B < 1 || a->Hq < 1 || a->Hkv < 1 || a->N < 1 || a->d < 1 || a->S < 1 ||
+        a->W < 1 || a->K < 1 || !a->head_map)
+        return HILS_ERR_INVALID_ARG;
+    if (a->Hq % a->Hkv) return HILS_ERR_INVALID_ARG;
+    if (a->K > HILS_MAX_TOPK || a->Hq > kMaxHeads) return HILS_ERR_UNSUPPORTED;
+    const int G = a->Hq / a->Hkv;
+    if (G > 8 || !(a->d == 64 || a->d == 128) || a->S != 64) return HILS_ERR_UNSUPPORTED;
+    if ((int64_t)a->B * a->Hq * a->N * a->d >= (1ll << 40)) return HILS_ERR_UNSUPPORTED;
+    int count[kMaxHeads];
+    for (int g = 0; g < a->Hkv; ++g) count[g] = 0;
+    for (int h = 0; h < a->Hq; ++h) {
+        const int g = a->head_map[h];
+        if (g < 0 || g >= a->Hkv || count[g] >= G) return HILS_ERR_INVALID_ARG;
+        p->group_heads[g * G + count[g]] = (int16_t)h;
+        count[g]++;
+    }
+    p->B = a->B; p->Hq = a->Hq; p->Hkv = a->Hkv; p->G = G; p->N = a->N;
+    p->S = a->S; p->W = a->W; p->K = a->K; p->nC = a->N / a->S;
+    p->inv_sqrt_d = (float)(1.0 / sqrt((double)a->d));
+    const size_t rows = (size_t)a->B * a->Hq * a->N;
+    const size_t need = (rows * 2 + rows * (size_t)a->K * 3) * sizeof(float);
+    if (ws_bytes) *ws_bytes = need;
+    if (!need_ptrs) return HILS_OK;
+    if (!a->Q || !a->Kc || !a->V || !a->dO || !a->idx || !a->dQ || !a->dK || !a->dV)
+        return HILS_ERR_INVALID_ARG;
+    if (p->nC > 0 && (!a->Klm || !a->bias || !a->dKlm || !a->dbias))
+        return HILS_ERR_INVALID_ARG;
+    if ((a->Qs != nullptr) != (a->dQs != nullptr)) return HILS_ERR_INVALID_ARG;
+    if (!a->workspace) return HILS_ERR_INVALID_ARG;
+    if (a->workspace_bytes < need) return HILS_ERR_WORKSPACE_TOO_SMALL;
+    const void *ptrs[] = {a->Q, a->Qs, a->Kc, a->V, a->Klm, a->bias, a->dO, a->idx,
+                          a->dQ, a->dQs, a->dK, a->dV, a->dKlm, a->dbias, a->workspace};
+    for (const void *q : ptrs)
+        if (q && !al16b(q)) return HILS_ERR_MISALIGNED;
+    p->Q = a->Q; p->Qs = a->Qs; p->Kc = a->Kc; p->Vc = a->V; p->Klm = a->Klm;
+    p->dO = a->dO; p->bias = a->bias; p->idx = a->idx;
+    p->dQ = a->dQ; p->dQs = a->dQs; p->dK = a->dK; p->dV = a->dV;
+    p->dKlm = a->dKlm; p->dbias = a->dbias;
+    p->rowstat = (float *)a->workspace;
+    p->chunkstat = p->rowstat + rows * 2;
+    return HILS_OK;
+}
+
+}  // namespace
+}  // namespace hils
+
+extern "C" hils_status hils_bwd_prefill_workspace_size(const hils_backward_args *a,
+                                                       size_t *bytes) {
+    using namespace hils;
+    if (!bytes) return HILS_ERR_INVALID_ARG;
+    BwdParams p;
+    size_t n = 0;
+    hils_status s = bwd_problem(a, &p, false, &n);
+    if (s != HILS_OK) return s;
+    *bytes = n;
+    return HILS_OK;
+}
+
+extern "C" hils_status hils_bwd_prefill(const hils_backward_args *a, void *stream) {
+    using namespace hils;
+    BwdParams p;
+    hils_status s = bwd_problem(a, &p, true, nullptr);
+    if (s != HILS_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (a->dtype == HILS_BF16)
+        e = a->d == 128 ? launch_bwd_d<__nv_bfloat16, 128>(p, st)
+                        : launch_bwd_d<__nv_bfloat16, 64>(p, st);
+    else
+        e = a->d == 128 ? launch_bwd_d<float, 128>(p, st)
+                        : launch_bwd_d<float, 64>(p, st);
+    count_launches(2);
+    return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
+}

@@ -268,6 +268,44 @@ hils_status hils_decode_multi_workspace_size(const hils_decode_multi_args *args,
 hils_status hils_fwd_decode_multi(const hils_decode_multi_args *args, void *stream);
 
 /*
+ * Backward of the prefill forward, for a fixed selection ("Hierarchical
+ * Sparse Attention Done Right", Sec. 3, RQ2: the fused chunk-level softmax
+ * lets the loss reach the landmark scores; Sec. 4, native sparse training).
+ * The top-K choice is discrete and held fixed; gradients of sum(O * dO) flow
+ * to Q, the scoring query, K, V, the landmark keys and the biases through
+ * the intra-chunk softmax, the chunk scores s^ and the window softmax.
+ *   Q, Qs, dO [B,Hq,N,d]; Kc, V [B,Hkv,N,d]; Klm [B,Hkv,nC,d]; bias
+ *   [B,Hkv,nC] f32; idx [B,Hkv,N,K] int32 (the forward's selection:
+ *   ascending, -1 padded; entries outside C_i are ignored, as the forward
+ *   ignores them); dtype of Q, Qs, dO, Kc, V, Klm: f32 or bf16.
+ *   Outputs, f32, overwritten (not accumulated): dQ [B,Hq,N,d], dQs (must be
+ *   given exactly when Qs is; without Qs the scoring gradient is in dQ), dK,
+ *   dV [B,Hkv,N,d], dKlm [B,Hkv,nC,d], dbias [B,Hkv,nC].
+ *   workspace >= hils_bwd_prefill_workspace_size (per (row, head) and
+ *   (row, head, selected chunk) softmax statistics).
+ * Deterministic: no floating-point atomics; every output element is summed
+ * by one thread in a fixed order. Supported: d in {64,128}, S = 64,
+ * G = Hq/Hkv <= 8; other shapes return HILS_ERR_UNSUPPORTED. Two kernel
+ * launches on `stream`.
+ */
+typedef struct {
+    int32_t dtype;
+    int32_t B, Hq, Hkv, N, d, S, W, K;
+    const int32_t *head_map;        /* host [Hq] */
+    const void *Q, *Qs, *Kc, *V, *Klm;
+    const float *bias;
+    const void *dO;
+    const int32_t *idx;
+    float *dQ, *dQs, *dK, *dV, *dKlm, *dbias;
+    void *workspace;
+    size_t workspace_bytes;
+} hils_backward_args;
+
+hils_status hils_bwd_prefill_workspace_size(const hils_backward_args *args,
+                                            size_t *bytes);
+hils_status hils_bwd_prefill(const hils_backward_args *args, void *stream);
+
+/*
  * Landmark summaries of the chunks: the (k', b') inputs of the scoring step.
  * "Hierarchical Sparse Attention Done Right", Sec. 3 (answering RQ1, the
  * surrogate of Eq. 7): for every full chunk c (nC = floor(N/S) of them) of

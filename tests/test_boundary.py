@@ -267,3 +267,32 @@ def test_decode_multi_validation(L):
     d.base.dtype = hils.F32               # no f32 multi-token kernels
     assert L.hils_fwd_decode_multi(ctypes.byref(d), None) == 2
     assert L.hils_fwd_decode_multi(None, None) == 1
+
+
+def _bwd(**kw):
+    fake = 1 << 40
+    hm = (ctypes.c_int32 * 8)(*[h // 4 for h in range(8)])
+    a = dict(dtype=hils.BF16, B=1, Hq=8, Hkv=2, N=1024, d=128, S=64, W=128,
+             K=8, head_map=ctypes.cast(hm, ctypes.c_void_p).value, Q=fake,
+             Qs=None, Kc=fake, V=fake, Klm=fake, bias=fake, dO=fake, idx=fake,
+             dQ=fake, dQs=None, dK=fake, dV=fake, dKlm=fake, dbias=fake,
+             workspace=fake, workspace_bytes=1 << 40)
+    a.update(kw)
+    return hils.BackwardArgs(**a), hm
+
+
+def test_backward_validation(L):
+    """Backward records are checked on the host before any launch (only
+    failing records reach the compute entry point)."""
+    a, hm = _bwd()
+    n = ctypes.c_size_t(0)
+    assert L.hils_bwd_prefill_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert n.value == 4 * (1 * 8 * 1024 * 2 + 1 * 8 * 1024 * 8 * 3)
+    fake = 1 << 40
+    for kw, code in [(dict(S=128), 2), (dict(d=96), 2), (dict(K=65), 2),
+                     (dict(dQ=None), 1), (dict(Qs=fake), 1),
+                     (dict(workspace_bytes=16), 4), (dict(dK=fake + 8), 3),
+                     (dict(Hkv=3), 1), (dict(dtype=5), 1)]:
+        b, hm2 = _bwd(**kw)
+        assert L.hils_bwd_prefill(ctypes.byref(b), None) == code, kw
+    assert L.hils_bwd_prefill(None, None) == 1

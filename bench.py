@@ -601,6 +601,8 @@ def main():
             peaks)
         line["landmarks"] = bench_landmarks(args, dev, stream, flush,
                                             max_over_ranks, barrier, peaks)
+        line["backward"] = bench_backward(args, dev, stream, flush,
+                                          max_over_ranks, barrier, rank)
 
     if rank == 0 and world == 1 and not args.no_cpu:
         cinp = synth.make_prefill(sh, seed=synth.seed_for(cfg_id),
@@ -756,6 +758,91 @@ def bench_decode(args, dev, stream, flush, world, max_over_ranks, barrier,
     del inp, O, idx, sel, ws
     torch.cuda.empty_cache()
     return out
+
+
+def fp32_alu_peak_tflops():
+    """FP32 FMA peak of the CUDA cores from unit counts and clocks: SMs x 128
+    FP32 lanes x 2 FLOP per FMA x the maximum SM clock."""
+    import torch
+    props = torch.cuda.get_device_properties(torch.cuda.current_device())
+    mhz = 1965.0
+    try:
+        import pynvml as nv
+        nv.nvmlInit()
+        h = nv.nvmlDeviceGetHandleByIndex(0)
+        mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+    except Exception:
+        pass
+    return props.multi_processor_count * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def bench_backward(args, dev, stream, flush, max_over_ranks, barrier, rank):
+    """Backward of the 32K prefill workload (selection from the forward,
+    dO ~ N(0,1)), L2 flushed before every call. The kernels run on the CUDA
+    cores in f32: roofline "alu" against the FP32 FMA peak, on the touched
+    FLOPs: 10d per (row, head, attended token) -- s, u, dq, dK, dV -- plus
+    4d per (row, head, selected chunk) for dqs and dk'."""
+    import torch
+
+    import chunk_sparse_long_landmark_b200 as hils
+    import synth
+    cid = WORKLOADS["prefill_32k"]
+    sh = synth.PREFILL_CONFIGS[cid]
+    inp = synth.make_prefill(sh, seed=synth.seed_for(cid) + 17 * rank + 3,
+                             device=dev)
+    _, idx = hils.fwd_prefill(inp["Q"], inp["K"], inp["V"], inp["Klm"],
+                              inp["bias"], inp["head_map"], sh.S, sh.W, sh.K,
+                              stream=stream)
+    g0 = torch.Generator(device=dev).manual_seed(11)
+    dO = torch.randn(inp["Q"].shape, generator=g0, device=dev).to(inp["Q"].dtype)
+    grads = None
+
+    def call():
+        nonlocal grads
+        grads = hils.bwd_prefill(inp["Q"], inp["K"], inp["V"], inp["Klm"],
+                                 inp["bias"], inp["head_map"], sh.S, sh.W,
+                                 idx, dO, grads=grads, stream=stream)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        call()
+    steps = max(1, min(args.steps, 3))
+    evs = [(torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    barrier()
+    torch.cuda.synchronize()
+    for a, b in evs:
+        flush.zero_()
+        a.record(stream)
+        call()
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in evs)) / steps
+    i = np.arange(sh.N, dtype=np.int64)
+    lq = np.floor_divide(i - sh.W + 1, sh.S)
+    nc = np.maximum(lq, 0)
+    w0 = np.maximum(lq * sh.S, 0)
+    sel = np.minimum(nc, sh.K)
+    toks = sel * sh.S + (i - w0 + 1)
+    flops = float(sh.B * sh.Hq * sh.d * (10 * toks.sum() + 4 * sel.sum()))
+    ach = flops / (ms * 1e-3) / 1e12
+    peak = fp32_alu_peak_tflops()
+    del inp, idx, dO, grads
+    torch.cuda.empty_cache()
+    return {"workload": "prefill_32k_backward",
+            "description": "dQ, dK, dV, dk', db' of the 32K prefill for the "
+                           "forward's selection",
+            "value": sh.B * sh.N / (ms * 1e-3), "unit": "tokens/s",
+            "ms_per_step": ms, "steps": steps,
+            "roofline": {"bound": "alu", "achieved": ach, "peak": peak,
+                         "unit": "TFLOP/s", "frac": ach / peak,
+                         "peak_source": "SMs x 128 FP32 lanes x 2 x max SM clock",
+                         "algorithmic_flops_per_call": flops,
+                         "traffic": None},
+            "config": {"B": sh.B, "Hq": sh.Hq, "Hkv": sh.Hkv, "d": sh.d,
+                       "N": sh.N, "S": sh.S, "W": sh.W, "K": sh.K,
+                       "dtype": "bf16 inputs, f32 arithmetic and gradients",
+                       "l2": "flushed before every call"}}
 
 
 DECODE_MULTI_T = 4

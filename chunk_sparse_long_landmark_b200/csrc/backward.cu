@@ -24,7 +24,7 @@
 //   bwd_keys  one CTA per (b, g, chunk of S tokens): the query rows that
 //             selected the chunk (found by scanning idx, ascending) and the
 //             rows whose window covers it, in ascending order; thread
-//             (token, quarter of dims) keeps its K/V slice and its dK/dV
+//             (token, eighth of dims) keeps its K/V slice and its dK/dV
 //             accumulators in registers. Also dk'_c and db'_c.
 // Inputs f32 or bf16, arithmetic and outputs f32.
 #include <math.h>
@@ -78,22 +78,52 @@ struct RowSmem {
     float sh[GM][HILS_MAX_TOPK], lz[GM][HILS_MAX_TOPK], ub[GM][HILS_MAX_TOPK];
 };
 
-// s = q_h . k_j and u = dO_h . v_j for the G heads, one token per lane.
+// 16 bytes of a row as f32: 8 bf16 or 4 f32 values
+__device__ __forceinline__ void unpack16(const uint4 &w, const __nv_bfloat16 *, float *f) {
+    const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        f[2 * k] = __uint_as_float(x[k] << 16);
+        f[2 * k + 1] = __uint_as_float(x[k] & 0xffff0000u);
+    }
+}
+__device__ __forceinline__ void unpack16(const uint4 &w, const float *, float *f) {
+    f[0] = __uint_as_float(w.x); f[1] = __uint_as_float(w.y);
+    f[2] = __uint_as_float(w.z); f[3] = __uint_as_float(w.w);
+}
+
+// s = q_h . k_j and u = dO_h . v_j for the G heads, one token per lane:
+// the token's rows in 16-byte loads, q and dO as float4 broadcasts from
+// shared memory.
 template <typename T, int D, int GM>
 __device__ __forceinline__ void token_dots(const RowSmem<D, GM> &sm, int G,
                                            const T *krow, const T *vrow,
                                            float *s, float *u) {
+    constexpr int E = 16 / (int)sizeof(T);
 #pragma unroll
     for (int h = 0; h < GM; ++h) s[h] = u[h] = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < D; ++k) {
-        const float kv = ld_f(krow + k), vv = ld_f(vrow + k);
+#pragma unroll 2
+    for (int k0 = 0; k0 < D; k0 += E) {
+        float kf[E], vf[E];
+        unpack16(__ldg(reinterpret_cast<const uint4 *>(krow + k0)), krow, kf);
+        unpack16(__ldg(reinterpret_cast<const uint4 *>(vrow + k0)), vrow, vf);
 #pragma unroll
-        for (int h = 0; h < GM; ++h)
-            if (h < G) {
-                s[h] = fmaf(sm.q[h][k], kv, s[h]);
-                u[h] = fmaf(sm.go[h][k], vv, u[h]);
+        for (int h = 0; h < GM; ++h) {
+            if (h >= G) break;
+#pragma unroll
+            for (int e4 = 0; e4 < E; e4 += 4) {
+                const float4 q4 = *reinterpret_cast<const float4 *>(&sm.q[h][k0 + e4]);
+                const float4 g4 = *reinterpret_cast<const float4 *>(&sm.go[h][k0 + e4]);
+                s[h] = fmaf(q4.x, kf[e4], s[h]);
+                s[h] = fmaf(q4.y, kf[e4 + 1], s[h]);
+                s[h] = fmaf(q4.z, kf[e4 + 2], s[h]);
+                s[h] = fmaf(q4.w, kf[e4 + 3], s[h]);
+                u[h] = fmaf(g4.x, vf[e4], u[h]);
+                u[h] = fmaf(g4.y, vf[e4 + 1], u[h]);
+                u[h] = fmaf(g4.z, vf[e4 + 2], u[h]);
+                u[h] = fmaf(g4.w, vf[e4 + 3], u[h]);
             }
+        }
     }
 }
 
@@ -322,11 +352,19 @@ bwd_rows_kernel(const BwdParams p) {
 }
 
 // ------------------------------------------------------------------ keys
-constexpr int kKeyBatch = 8;                     // (row, head) pairs per round
+constexpr int kKeyBatch = 16;                    // (row, head) pairs per round
+constexpr int kKeySplit = 8;                     // threads per token
+
+// A pair's q / dO / qs row is stored as kKeySplit slices of D/kKeySplit
+// floats, each padded by 4: the 8 threads of a token read their slices as
+// float4 from 8 disjoint bank groups (slice stride 80 or 48 bytes).
+template <int D>
+constexpr int kSlice = D / kKeySplit + 4;
 
 template <int D, int GM>
 struct KeySmem {
-    float q[kKeyBatch][D], go[kKeyBatch][D], qs[kKeyBatch][D];
+    float q[kKeyBatch][kKeySplit][kSlice<D>], go[kKeyBatch][kKeySplit][kSlice<D>],
+          qs[kKeyBatch][kKeySplit][kSlice<D>];
     // per pair: chunk role (lz, P, Ubar), window role (L, D, -); the row's
     // token range inside the chunk; dsh = P (Ubar - D) (chunk role)
     float a0[kKeyBatch], a1[kKeyBatch], a2[kKeyBatch], dsh[kKeyBatch];
@@ -339,10 +377,10 @@ struct KeySmem {
 };
 
 template <typename T, int D, int S_TOK, int GM>
-__global__ void __launch_bounds__(S_TOK * 4)
+__global__ void __launch_bounds__(S_TOK * kKeySplit)
 bwd_keys_kernel(const BwdParams p) {
-    constexpr int DQ = D / 4;                    // dims per thread
-    constexpr int NT = S_TOK * 4;
+    constexpr int DQ = D / kKeySplit;            // dims per thread
+    constexpr int NT = S_TOK * kKeySplit;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     KeySmem<D, GM> &sm = *reinterpret_cast<KeySmem<D, GM> *>(smem_raw);
     const int nchunks = (p.N + S_TOK - 1) / S_TOK;
@@ -350,7 +388,7 @@ bwd_keys_kernel(const BwdParams p) {
     const int g = (blockIdx.x / nchunks) % p.Hkv;
     const int b = blockIdx.x / (nchunks * p.Hkv);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int jl = tid >> 2, qd = tid & 3;
+    const int jl = tid / kKeySplit, qd = tid % kKeySplit;
     const int64_t j = (int64_t)c * S_TOK + jl;   // this thread's token
     const bool jok = j < p.N;
     const int G = p.G;
@@ -386,9 +424,9 @@ bwd_keys_kernel(const BwdParams p) {
                 const int hq = p.group_heads[g * G + h];
                 const int64_t rq = ((int64_t)b * p.Hq + hq) * p.N + ri;
                 for (int k = lane; k < D; k += 32) {
-                    sm.q[e][k] = ld_f(Qp + rq * D + k);
-                    sm.go[e][k] = ld_f(dOp + rq * D + k);
-                    if (role == 0) sm.qs[e][k] = ld_f(Qsp + rq * D + k);
+                    sm.q[e][k / DQ][k % DQ] = ld_f(Qp + rq * D + k);
+                    sm.go[e][k / DQ][k % DQ] = ld_f(dOp + rq * D + k);
+                    if (role == 0) sm.qs[e][k / DQ][k % DQ] = ld_f(Qsp + rq * D + k);
                 }
                 if (lane == 0) {
                     if (role == 0) {             // lz, P, Ubar and D of the row
@@ -412,16 +450,29 @@ bwd_keys_kernel(const BwdParams p) {
             }
             __syncthreads();
             for (int e = 0; e < ne; ++e) {       // fixed order: deterministic
+                const float4 *q4p = reinterpret_cast<const float4 *>(&sm.q[e][qd][0]);
+                const float4 *g4p = reinterpret_cast<const float4 *>(&sm.go[e][qd][0]);
+                float4 q4[DQ / 4], g4[DQ / 4];
+#pragma unroll
+                for (int r = 0; r < DQ / 4; ++r) { q4[r] = q4p[r]; g4[r] = g4p[r]; }
                 float sp = 0.f, up = 0.f;
 #pragma unroll
-                for (int r = 0; r < DQ; ++r) {
-                    sp = fmaf(sm.q[e][qd * DQ + r], kreg[r], sp);
-                    up = fmaf(sm.go[e][qd * DQ + r], vreg[r], up);
+                for (int r = 0; r < DQ / 4; ++r) {
+                    const float4 a = q4[r], c4 = g4[r];
+                    sp = fmaf(a.x, kreg[4 * r], sp);
+                    sp = fmaf(a.y, kreg[4 * r + 1], sp);
+                    sp = fmaf(a.z, kreg[4 * r + 2], sp);
+                    sp = fmaf(a.w, kreg[4 * r + 3], sp);
+                    up = fmaf(c4.x, vreg[4 * r], up);
+                    up = fmaf(c4.y, vreg[4 * r + 1], up);
+                    up = fmaf(c4.z, vreg[4 * r + 2], up);
+                    up = fmaf(c4.w, vreg[4 * r + 3], up);
                 }
-                sp += __shfl_xor_sync(0xffffffffu, sp, 1);
-                up += __shfl_xor_sync(0xffffffffu, up, 1);
-                sp += __shfl_xor_sync(0xffffffffu, sp, 2);
-                up += __shfl_xor_sync(0xffffffffu, up, 2);
+#pragma unroll
+                for (int o = 1; o < kKeySplit; o <<= 1) {   // the token's threads
+                    sp += __shfl_xor_sync(0xffffffffu, sp, o);
+                    up += __shfl_xor_sync(0xffffffffu, up, o);
+                }
                 const float x = sp * isd;
                 float pj = 0.f, dsj = 0.f;
                 if (jok && jl >= sm.lo[e] && jl <= sm.hi[e]) {
@@ -434,15 +485,22 @@ bwd_keys_kernel(const BwdParams p) {
                     }
                 }
 #pragma unroll
-                for (int r = 0; r < DQ; ++r) {
-                    adv[r] = fmaf(pj, sm.go[e][qd * DQ + r], adv[r]);
-                    adk[r] = fmaf(dsj, sm.q[e][qd * DQ + r], adk[r]);
+                for (int r = 0; r < DQ / 4; ++r) {
+                    const float4 a = q4[r], c4 = g4[r];
+                    adv[4 * r] = fmaf(pj, c4.x, adv[4 * r]);
+                    adv[4 * r + 1] = fmaf(pj, c4.y, adv[4 * r + 1]);
+                    adv[4 * r + 2] = fmaf(pj, c4.z, adv[4 * r + 2]);
+                    adv[4 * r + 3] = fmaf(pj, c4.w, adv[4 * r + 3]);
+                    adk[4 * r] = fmaf(dsj, a.x, adk[4 * r]);
+                    adk[4 * r + 1] = fmaf(dsj, a.y, adk[4 * r + 1]);
+                    adk[4 * r + 2] = fmaf(dsj, a.z, adk[4 * r + 2]);
+                    adk[4 * r + 3] = fmaf(dsj, a.w, adk[4 * r + 3]);
                 }
             }
             if (role == 0) {                     // k' and b' of the chunk
                 for (int k = tid; k < D; k += NT) {
                     float a = sm.dklm[k];
-                    for (int e = 0; e < ne; ++e) a = fmaf(sm.dsh[e], sm.qs[e][k], a);
+                    for (int e = 0; e < ne; ++e) a = fmaf(sm.dsh[e], sm.qs[e][k / DQ][k % DQ], a);
                     sm.dklm[k] = a;
                 }
                 if (tid == NT - 1) {
@@ -551,7 +609,7 @@ cudaError_t launch_keys_t(const BwdParams &p, cudaStream_t st) {
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = (int64_t)p.B * p.Hkv * ((p.N + S_TOK - 1) / S_TOK);
-    bwd_keys_kernel<T, D, S_TOK, GM><<<(unsigned)grid, S_TOK * 4, smem, st>>>(p);
+    bwd_keys_kernel<T, D, S_TOK, GM><<<(unsigned)grid, S_TOK * kKeySplit, smem, st>>>(p);
     return cudaGetLastError();
 }
 

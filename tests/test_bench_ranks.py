@@ -61,3 +61,33 @@ def test_single_process_needs_no_process_group():
     assert ctx.max(3.5) == 3.5
     assert ctx.whole_job_rate(500, 5.0) == pytest.approx(1e5)
     ctx.close()
+
+
+def test_decode_multi_bytes_reduces_to_single_token():
+    """The multi-token bytes model with T = 1 is the decode bytes model, and
+    tokens that share every chunk add only their Q / O / idx bytes."""
+    import numpy as np
+
+    import bench
+    import synth
+    sh = synth.Shape("bf16", 2, 8, 2, 128, 8192, 64, 512, 4)
+    cl = [8192, 5000]
+    rng = np.random.default_rng(0)
+    idx1 = np.full((2, 1, 2, 4), -1, dtype=np.int64)
+    for b, L in enumerate(cl):
+        nc = (L - 1 - sh.W + 1) // sh.S
+        for g in range(2):
+            idx1[b, 0, g] = np.sort(rng.choice(nc, 4, replace=False))
+    assert bench.decode_multi_bytes(sh, cl, 1, idx1) == bench.decode_bytes(sh, cl)
+    # two tokens (positions L-2, L-1) with the same selection: the chunks and
+    # the landmark scan are shared; the window union reaches back to the
+    # earlier token's window start; each token adds its Q / O / idx bytes
+    idx2 = np.repeat(idx1, 2, axis=1)
+    extra = bench.decode_multi_bytes(sh, cl, 2, idx2) - bench.decode_bytes(sh, cl)
+    esz = 2
+    want = 0
+    for L in cl:
+        w0 = lambda i: max((i - sh.W + 1) // sh.S * sh.S, 0)
+        want += (w0(L - 1) - w0(L - 2)) * sh.Hkv * 2 * sh.d * esz
+        want += 2 * sh.Hq * sh.d * esz + sh.Hkv * sh.K * 4
+    assert extra == want

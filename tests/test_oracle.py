@@ -346,3 +346,28 @@ def test_oracle_bf16_storage_widens_exactly():
     r32 = oracle.prefill_full(inp32)
     np.testing.assert_array_equal(r16["idx"], r32["idx"])
     np.testing.assert_array_equal(r16["O"], r32["O"])
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_group_topk_lies_in_union_of_per_split_per_head_topk(seed):
+    """The group top-K (a_c = max_h (s^_hc - LSE_h), ties to the lower
+    chunk) is contained in the union, over contiguous splits of the
+    candidates and over heads, of each split's per-head top-K by s^ (same
+    tie rule): a chunk outside its split's top-K for its maximising head has
+    K chunks of that split ranked above it for every head's offset. This
+    bounds what a split-local pre-selection may discard. Exact ties are
+    planted so the tie rule is exercised."""
+    r = np.random.default_rng(seed)
+    G, nc, K = 4, 300, 16
+    shat = np.round(r.standard_normal((G, nc)) * 4) / 4      # many exact ties
+    idx, _ = brute.select(shat[:, None, :], np.array([nc]), K)
+    chosen = set(int(c) for c in idx[0] if c >= 0)
+    for nsplit in (1, 3, 7, 19):
+        bounds_ = np.linspace(0, nc, nsplit + 1).astype(int)
+        union = set()
+        for a, b in zip(bounds_[:-1], bounds_[1:]):
+            for h in range(G):
+                c = np.arange(a, b)
+                order = np.lexsort((c, -shat[h, a:b]))
+                union.update(int(x) for x in c[order[:K]])
+        assert chosen <= union, (nsplit, sorted(chosen - union))

@@ -8,10 +8,12 @@ One step = one HiLS prefill forward (landmark scoring + group top-K +
 gathered intra-chunk/window attention + chunk-softmax fusion) over the
 workload's whole synthetic input, through the C ABI (hils_prefill_select then
 hils_prefill_attend, exactly what hils_fwd_prefill runs), inputs resident in
-HBM. The default workload is the 32K prefill (B=1, Hq=32, Hkv=8, d=128,
-S=64, W=512, K=16, planted needles). The decode step of the 512K, batch-8
-workload is measured in the same run (as a CUDA graph) and reported under
-"decode". L2 is flushed (256 MiB write) before every timed step.
+HBM. The headline workload is the 512K prefill (B=1, Hq=32, Hkv=8, d=128,
+S=128, W=2048, K=32, planted needles every 64K tokens); the 128K and 32K
+prefills follow as their own legs ("prefill_128k", "prefill_32k"), each
+with its roofline. The decode step of the 512K, batch-8 workload is measured
+in the same run (as a CUDA graph) and reported under "decode". L2 is flushed
+(256 MiB write) before every timed step.
 
 Rank 0 prints one JSON line. Under torchrun each rank runs its own replica of
 the workload on its own GPU (the path shards by (batch, kv head) with no
@@ -41,6 +43,9 @@ METRIC = ("HiLS fwd prefill tokens/s & decode µs/token at 1 B200; "
 WORKLOADS = {"prefill_32k": 2, "prefill_128k": 3, "prefill_512k": 5}
 DECODE_WORKLOAD = ("decode_512k_b8", 4)
 L2_FLUSH_BYTES = 256 << 20
+# query positions per oracle batch (each evaluated for every kv group): 16
+# positions x 8 groups keep 16 host cores busy in one batch
+REF_POSITIONS = 16
 
 
 # ------------------------------------------------------------ work counting
@@ -301,15 +306,16 @@ def profiled_traffic(kernels, workload):
 
 
 # -------------------------------------------------------------- oracle arm
-def oracle_sample(inp, budget_s, positions_per_batch=8, seed=0,
-                  max_batches=None):
+def oracle_sample(inp, budget_s, positions_per_batch=REF_POSITIONS, seed=0,
+                  max_batches=None, bound=None):
     """Time the fp64 oracle on random query positions of the workload until
     `budget_s` seconds of work. Returns (tokens/s, positions, seconds,
-    threads)."""
+    threads). `bound`: the inputs already copied to the host by
+    oracle.bind_prefill (copied here otherwise, outside the timing)."""
     import oracle
     sh = inp["shape"]
     rng = np.random.default_rng(seed)
-    bound = oracle.bind_prefill(inp)
+    bound = bound or oracle.bind_prefill(inp)
     done, t0 = 0, time.perf_counter()
     nb = 0
     while True:
@@ -340,14 +346,20 @@ def run_reference(args, sh, name):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
+    import torch
+    # the inputs are drawn on the GPU when there is one (the same numbers as
+    # the GPU arm's) and copied to the host by the oracle's binding
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
     inp = synth.make_prefill(sh, seed=synth.seed_for(WORKLOADS[name]),
-                             device="cpu")
+                             device=dev)
+    import oracle
+    bound = oracle.bind_prefill(inp)
     per_step = []
     cnt = []
     for s in range(args.warmup + args.steps):
         v, n, el, thr = oracle_sample(inp, budget_s=0.0,
-                                      positions_per_batch=4, seed=s,
-                                      max_batches=1)
+                                      positions_per_batch=REF_POSITIONS,
+                                      seed=s, max_batches=1, bound=bound)
         if s >= args.warmup:
             per_step.append(el)
             cnt.append(n)
@@ -362,7 +374,8 @@ def run_reference(args, sh, name):
         "config": workload_config(sh, name),
         "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": thr,
                          "kind": "oracle",
-                         "sample": f"4 random query positions (all heads) "
+                         "sample": f"{REF_POSITIONS} random query positions "
+                                   f"x {sh.Hkv} kv groups (all {sh.Hq} heads) "
                                    f"per step of the {name} workload"},
         "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -426,65 +439,33 @@ class RankContext:
 
 
 # ---------------------------------------------------------------- GPU arm
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="prefill_32k",
-                    choices=sorted(WORKLOADS))
-    ap.add_argument("--impl", default="hils", choices=["hils", "reference"])
-    ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--decode-only", action="store_true",
-                    help="time only the decode step (prints its object)")
-    args = ap.parse_args()
-    args.warmup = max(args.warmup, 3)
+def bench_prefill(args, name, dev, stream, flush, ranks, peaks, steps,
+                  with_e2e, rank):
+    """Time one prefill workload through the C ABI (select then attend, as
+    hils_fwd_prefill runs them), L2 flushed before every timed step.
 
-    import synth
-    cfg_id = WORKLOADS[args.workload]
-    sh = synth.PREFILL_CONFIGS[cfg_id]
-    if args.impl == "reference":
-        run_reference(args, sh, args.workload)
-        return
-
+    Returns the leg's dict: step time, stage times, the dominant kernel's
+    roofline (algorithmic FLOPs of that stage / its mean event-timed
+    duration), the whole step's fraction on the touched FLOPs of select +
+    attend, chunk-union diagnostics and, if asked, the end-to-end figure
+    (pinned host buffers, copies inside the timed region)."""
     import torch
 
     import chunk_sparse_long_landmark_b200 as hils
-
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    ranks = RankContext("nccl", dev)
-    world, rank = ranks.world, ranks.rank
-    barrier, max_over_ranks = ranks.barrier, ranks.max
-
-    peaks = measured_peaks()
-    if args.decode_only:
-        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-        d = bench_decode(args, dev, torch.cuda.current_stream(dev), flush,
-                         world, max_over_ranks, barrier, rank, peaks)
-        dm = bench_decode_multi(args, dev, torch.cuda.current_stream(dev),
-                                flush, world, max_over_ranks, barrier, rank,
-                                peaks)
-        if rank == 0:
-            print(json.dumps({"decode": d, "decode_multi": dm}), flush=True)
-        ranks.close()
-        return
+    import synth
+    cfg_id = WORKLOADS[name]
+    sh = synth.PREFILL_CONFIGS[cfg_id]
     inp = synth.make_prefill(sh, seed=synth.seed_for(cfg_id) + 17 * rank,
                              device=dev)
     work = prefill_work(sh)
-    B, Hq, Hkv, N, d, K = sh.B, sh.Hq, sh.Hkv, sh.N, sh.d, sh.K
+    B, Hq, Hkv, N, K = sh.B, sh.Hq, sh.Hkv, sh.N, sh.K
     O = torch.empty_like(inp["Q"])
     idx = torch.empty(B, Hkv, N, K, dtype=torch.int32, device=dev)
     sel = torch.empty(B, Hq, N, K, dtype=torch.float32, device=dev)
-    ws = torch.empty(hils.prefill_workspace_size(
+    ws = torch.empty(max(1, hils.prefill_workspace_size(
         inp["Q"], inp["K"], inp["V"], inp["Klm"], inp["bias"],
-        inp["head_map"], sh.S, sh.W, K, with_sel_score=True),
+        inp["head_map"], sh.S, sh.W, K, with_sel_score=True)),
         dtype=torch.uint8, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
 
     def call(stage):
         hils.fwd_prefill(inp["Q"], inp["K"], inp["V"], inp["Klm"],
@@ -498,12 +479,12 @@ def main():
     torch.cuda.synchronize()
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
-           for _ in range(args.steps)]
-    barrier()
+           for _ in range(steps)]
+    ranks.barrier()
     torch.cuda.synchronize()
     n0 = hils.launch_count()
-    with ClockSampler(local) as clk:
-        for s in range(args.steps):
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for s in range(steps):
             flush.zero_()
             evs[s][0].record(stream)
             call("select")
@@ -511,48 +492,55 @@ def main():
             call("attend")
             evs[s][2].record(stream)
         torch.cuda.synchronize()
-    barrier()
+    ranks.barrier()
     launches = hils.launch_count() - n0
     t_sel = [e[0].elapsed_time(e[1]) for e in evs]
     t_att = [e[1].elapsed_time(e[2]) for e in evs]
     t_step = [a + b for a, b in zip(t_sel, t_att)]
-    tot_ms = max_over_ranks(sum(t_step))
-    ms_step = tot_ms / args.steps
+    ms_step = ranks.max(sum(t_step)) / steps
     value = ranks.whole_job_rate(work["tokens"], ms_step)
 
-    # dominant kernel roofline (tensor-bound contraction)
+    # a region of more than 2 s of back-to-back kernels runs under the power
+    # cap: it is compared with the sustained GEMM figure
+    sustained = steps * ms_step > 2000
+    peak = peaks["bf16_sustained"] if sustained else peaks["bf16"]
     a_ms, s_ms = statistics.mean(t_att), statistics.mean(t_sel)
     if a_ms >= s_ms:
         dom, dom_ms, dom_flops = "attend", a_ms, work["attend_flops"]
     else:
         dom, dom_ms, dom_flops = "select", s_ms, work["select_flops"]
     achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-    peak = peaks["bf16_sustained"] if args.steps * ms_step > 2000 else \
-        peaks["bf16"]
+    touched = work["select_flops"] + work["attend_flops"]
+    step_ach = touched / (ms_step * 1e-3) / 1e12
     roof = {"bound": "tensor", "kernel": dom, "achieved": achieved,
             "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-            "peak_source": peaks["src"],
+            "peak_source": peaks["src"] + (" (sustained bf16 GEMM)" if sustained
+                                           else " (burst bf16 GEMM)"),
             "algorithmic_flops_per_launch": dom_flops,
             "traffic": profiled_traffic(
-                ["tc_attend" if dom == "attend" else "tc_select"],
-                args.workload)}
+                ["tc_attend" if dom == "attend" else "tc_select"], name),
+            "whole_step": {
+                "achieved": step_ach, "frac": step_ach / peak,
+                "touched_flops": touched,
+                "definition": "touched FLOPs of scoring + intra-chunk + "
+                              "window attention (a2 + a5 + a6) / step time"},
+            "stages": {
+                "select": {"achieved": work["select_flops"] / (s_ms * 1e-3) / 1e12,
+                           "frac": work["select_flops"] / (s_ms * 1e-3) / 1e12 / peak,
+                           "flops": work["select_flops"]},
+                "attend": {"achieved": work["attend_flops"] / (a_ms * 1e-3) / 1e12,
+                           "frac": work["attend_flops"] / (a_ms * 1e-3) / 1e12 / peak,
+                           "flops": work["attend_flops"]}}}
+    leg = {"workload": name, "value": value, "unit": "tokens/s",
+           "ms_per_step": ms_step, "steps": steps,
+           "stages_ms": {"select": s_ms, "attend": a_ms},
+           "roofline": roof, "gpu_launches": int(launches),
+           "clocks": clk.summary(), "union": union_stats(sh, idx),
+           "config": workload_config(sh, name)}
 
-    line = {
-        "metric": METRIC, "value": value, "unit": "tokens/s",
-        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(sh, args.workload),
-        "stages_ms": {"select": s_ms, "attend": a_ms},
-        "roofline": roof,
-        "gpu_launches": int(launches),
-        "clocks": clk.summary(),
-        "union": union_stats(sh, idx),
-    }
-
-    # end to end through the C ABI with host buffers (pinned), per step:
-    # H2D of Q, K, V, Klm, bias; the call; D2H of O and idx
-    if not args.no_e2e:
+    if with_e2e:
+        # end to end through the C ABI with host buffers (pinned), per step:
+        # H2D of Q, K, V, Klm, bias; the call; D2H of O and idx
         host = host_inputs(inp)
         Oh = torch.empty(O.shape, dtype=O.dtype).pin_memory()
         Ih = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
@@ -573,25 +561,99 @@ def main():
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize()
-        barrier()
+        ranks.barrier()
         ee = [(torch.cuda.Event(enable_timing=True),
                torch.cuda.Event(enable_timing=True))
-              for _ in range(max(3, args.steps // 4))]
+              for _ in range(max(3, steps // 4))]
         for a, b in ee:
             flush.zero_()
             a.record(stream)
             e2e_step()
             b.record(stream)
         torch.cuda.synchronize()
-        e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ee)) / len(ee)
-        line["e2e"] = {"value": world * work["tokens"] / (e_ms * 1e-3),
-                       "unit": "tokens/s", "ms_per_step": e_ms,
-                       "h2d_bytes_per_step": int(h2d),
-                       "d2h_bytes_per_step": int(d2h)}
-        del host, dvs
-
+        e_ms = ranks.max(sum(a.elapsed_time(b) for a, b in ee)) / len(ee)
+        leg["e2e"] = {"value": ranks.world * work["tokens"] / (e_ms * 1e-3),
+                      "unit": "tokens/s", "ms_per_step": e_ms,
+                      "h2d_bytes_per_step": int(h2d),
+                      "d2h_bytes_per_step": int(d2h)}
+        del host, dvs, Oh, Ih
     del inp, O, idx, sel, ws
     torch.cuda.empty_cache()
+    return leg
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill_512k",
+                    choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="hils", choices=["hils", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-legs", action="store_true",
+                    help="skip the other prefill workloads' legs")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the decode step (prints its object)")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    import synth
+    cfg_id = WORKLOADS[args.workload]
+    sh = synth.PREFILL_CONFIGS[cfg_id]
+    if args.impl == "reference":
+        run_reference(args, sh, args.workload)
+        return
+
+    import torch
+
+    import chunk_sparse_long_landmark_b200 as hils  # noqa: F401 (fails loudly)
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    ranks = RankContext("nccl", dev)
+    world, rank = ranks.world, ranks.rank
+    barrier, max_over_ranks = ranks.barrier, ranks.max
+
+    peaks = measured_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    if args.decode_only:
+        d = bench_decode(args, dev, stream, flush, world, max_over_ranks,
+                         barrier, rank, peaks)
+        dm = bench_decode_multi(args, dev, stream, flush, world,
+                                max_over_ranks, barrier, rank, peaks)
+        if rank == 0:
+            print(json.dumps({"decode": d, "decode_multi": dm}), flush=True)
+        ranks.close()
+        return
+
+    head = bench_prefill(args, args.workload, dev, stream, flush, ranks,
+                         peaks, args.steps, not args.no_e2e, rank)
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": head["config"],
+        "stages_ms": head["stages_ms"], "roofline": head["roofline"],
+        "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+        "union": head["union"],
+    }
+    if "e2e" in head:
+        line["e2e"] = head["e2e"]
+
+    if not args.no_legs:
+        # the other prefill workloads, each with its own roofline
+        for other in sorted(WORKLOADS, key=lambda n: -WORKLOADS[n]):
+            if other == args.workload:
+                continue
+            line[other] = bench_prefill(args, other, dev, stream, flush, ranks,
+                                        peaks, max(args.steps, 10), False,
+                                        rank)
 
     if not args.no_decode:
         line["decode"] = bench_decode(args, dev, stream, flush, world,
@@ -607,11 +669,13 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu:
         cinp = synth.make_prefill(sh, seed=synth.seed_for(cfg_id),
                                   device=dev)
-        v, n, el, thr = oracle_sample(cinp, budget_s=15.0)
+        v, n, el, thr = oracle_sample(cinp, budget_s=15.0,
+                                      positions_per_batch=REF_POSITIONS)
         line["cpu_baseline"] = {
             "value": v, "unit": "tokens/s", "cores": thr, "kind": "oracle",
-            "sample": f"{n} random query positions (all {Hq} heads) of the "
-                      f"{args.workload} workload, {el:.1f} s"}
+            "sample": f"{n} random query positions (all {sh.Hq} heads, "
+                      f"{REF_POSITIONS} positions x {sh.Hkv} kv groups per "
+                      f"batch) of the {args.workload} workload, {el:.1f} s"}
         del cinp
 
     if rank == 0:

@@ -11,11 +11,15 @@
 //               dot-product engine: 16 chunks x 8 head slots x 16 dims),
 //               raw s^ -> workspace, per-split (max, sum-exp) per head.
 //   dec_select  one CTA per (b, kv head): merge the log-sum-exp partials,
-//               group score a_c = max_h (s^_hc - LSE_h), exact top-K by a
-//               4-round radix select (ties to the lower chunk), idx
-//               ascending, s^ of the selected chunks.
+//               group score a_c = max_h (s^_hc - LSE_h); a provable lower
+//               bound on the K-th best score (from each warp's two best)
+//               keeps K + a few candidates, ordered by a warp bitonic sort
+//               (ties to the lower chunk); longer lists get exact ranks
+//               counted in shared memory, and lists of more than 1024
+//               entries (mass ties) a radix select. idx ascending, s^ of
+//               the selected chunks.
 //   dec_attend  one CTA per (b, kv head, group of selected-chunk / window
-//               tiles), one wave in all: K/V tiles double-buffered by TMA,
+//               tiles), one wave in all: K/V tiles triple-buffered by TMA,
 //               QK^T and PV with mma.sync, intra-chunk softmax scaled by
 //               exp(s^_c) (chunk tiles) or plain masked softmax (window
 //               tiles), merged online -> partial (m, l, o) per group; the
@@ -691,7 +695,7 @@ dec_select_kernel(const DecParams p) {
 // -------------------------------------------------------------- dec_attend
 // One CTA = (b, kv head, group of kAttPer consecutive tiles of that (b, g)'s
 // tile list: the selected chunks in idx order, then the window tiles). The
-// CTA streams its tiles through a double-buffered TMA pipeline and merges
+// CTA streams its tiles through a triple-buffered TMA pipeline and merges
 // them online per head: running reference max M, O accumulated in the MMA
 // registers (rescaled when M rises), l in registers.
 constexpr int kAttPerMin = 4;                    // tiles per CTA, at least

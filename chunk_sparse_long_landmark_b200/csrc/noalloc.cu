@@ -11,9 +11,14 @@
 //
 // The array is a file-scope __device__ symbol. In host code its name is only
 // a host-side stand-in, not a device address, so the address is obtained
-// once per device with cudaGetSymbolAddress (with that device current) and
-// passed to the kernels as a plain pointer.
+// with cudaGetSymbolAddress (with the device current) on the first call in a
+// device's context and passed to the kernels as a plain pointer. The cached
+// address is keyed on the context's process-unique ID (cuCtxGetId): after a
+// cudaDeviceReset the library's module is loaded again in a new context,
+// where the array may sit elsewhere, and the address is looked up again.
 #include <mutex>
+
+#include <cuda.h>
 
 #include "hils_internal.cuh"
 
@@ -25,23 +30,61 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
 
-// Device address of the scratch array on the current device (set up on the
-// first call per device). Returns nullptr if the runtime refuses.
+struct CachedScratch {
+    unsigned long long ctx_id;      // context the address belongs to
+    void *ptr;
+};
+
+std::mutex g_mu;
+CachedScratch g_scratch[kMaxDevices] = {};
+
+// Unique ID of the calling thread's current context (false: none current,
+// or the driver entry points are unavailable).
+bool current_context_id(unsigned long long *id) {
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault,
+                                    &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = (CtxGetCurrentFn)f;
+        f = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault,
+                                    &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = (CtxGetIdFn)f;
+    });
+    CUcontext ctx = nullptr;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx)
+        return false;
+    return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array in the current device's context,
+// looked up on the first call in that context. nullptr if the runtime
+// refuses.
 void *scratch_for_current_device() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
         return nullptr;
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_scratch_ptr[dev]) {
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess)
-            return nullptr;
-        g_scratch_ptr[dev] = ptr;
-    }
-    return g_scratch_ptr[dev];
+    unsigned long long id = 0;
+    if (g_scratch[dev].ptr && current_context_id(&id) &&
+        id == g_scratch[dev].ctx_id)
+        return g_scratch[dev].ptr;
+    void *ptr = nullptr;           // (creates the primary context if needed)
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess)
+        return nullptr;
+    if (!current_context_id(&id)) return nullptr;
+    g_scratch[dev].ctx_id = id;
+    g_scratch[dev].ptr = ptr;
+    return ptr;
 }
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }

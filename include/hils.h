@@ -194,9 +194,12 @@ hils_status hils_decode_attend(const hils_decode_args *args, void *stream);
  * array inside the library (every GPU that loads the library holds it until
  * exit). It runs the CUDA-core decode kernels. The library allocates
  * nothing on this path.
- *   - The first call on a device, with that device current, looks up the
- *     array's device address (cudaGetSymbolAddress); make that first call
- *     before any stream capture.
+ *   - The first call in a device's context, with that device current, looks
+ *     up the array's device address (cudaGetSymbolAddress); make that first
+ *     call before any stream capture. The address is cached per device and
+ *     keyed on the context's process-unique ID, so after cudaDeviceReset (a
+ *     new context, where the array may sit elsewhere) the next call looks it
+ *     up again; make that call before any capture too.
  *   - Every call shares the one array and the next call overwrites it; calls
  *     whose executions overlap on the GPU (different streams, concurrent
  *     graphs) race on it. Nothing in it needs to start at zero.

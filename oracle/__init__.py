@@ -270,34 +270,45 @@ def decode(inp, score_mode=SCORE_LANDMARK, imposed_idx=None, threads=0,
 
 
 def prefill_at(inp, positions, score_mode=SCORE_LANDMARK, imposed_idx=None,
-               threads=0):
+               threads=0, groups=None, bound=None):
     """Oracle at chosen query positions of a (possibly huge) prefill problem.
 
     Only the Q / Qs rows at ``positions`` are copied to the host; K, V, Klm
-    and bias are copied whole. Returns per-(b, g, position) arrays shaped
-    O [B,Hkv,P,G,d], idx [B,Hkv,P,K], shat_sel [B,Hkv,P,G,K], gap/akth
-    [B,Hkv,P]. ``imposed_idx``: [B,Hkv,P,K] or None.
+    and bias are copied whole (or taken from ``bound``, a ``bind_at`` result
+    for the same positions). ``groups`` restricts the kv groups evaluated
+    (default: all, in order). Returns per-(b, g, position) arrays shaped
+    O [B,nG,P,G,d], idx [B,nG,P,K], shat_sel [B,nG,P,G,K], gap/akth
+    [B,nG,P], nG = len(groups). ``imposed_idx``: [B,nG,P,K] or None.
     """
-    import torch
     sh = inp["shape"]
     pos = np.asarray(positions, dtype=np.int64)
     P = len(pos)
-    pt = torch.as_tensor(pos, device=inp["Q"].device)
-    Qsub = inp["Q"].index_select(2, pt)
-    Qssub = inp["Qs"].index_select(2, pt) if inp.get("Qs") is not None \
-        else None
-    bd = _Bound(Qsub, Qssub, inp["K"], inp["V"], inp["Klm"], inp["bias"],
-                inp["head_map"], sh.S, sh.W, sh.K, q_rows=P)
-    bb, gg, pp = np.meshgrid(np.arange(sh.B), np.arange(sh.Hkv),
-                             np.arange(P), indexing="ij")
+    gs = np.arange(sh.Hkv) if groups is None else np.asarray(groups)
+    nG = len(gs)
+    bd = bound or bind_at(inp, pos)
+    bb, gg, pp = np.meshgrid(np.arange(sh.B), gs, np.arange(P), indexing="ij")
     rb, rg, rp = bb.ravel(), gg.ravel(), pp.ravel()
     imp = None
     if imposed_idx is not None:
         imp = np.asarray(imposed_idx, dtype=np.int32).reshape(-1, sh.K)
     r = bd.rows(rb, rg, pos[rp], rp, score_mode, imp, threads)
     G, d, K = sh.G, sh.d, sh.K
-    return dict(O=r["O"].reshape(sh.B, sh.Hkv, P, G, d),
-                idx=r["idx"].reshape(sh.B, sh.Hkv, P, K),
-                shat_sel=r["shat_sel"].reshape(sh.B, sh.Hkv, P, G, K),
-                gap=r["gap"].reshape(sh.B, sh.Hkv, P),
-                akth=r["akth"].reshape(sh.B, sh.Hkv, P))
+    return dict(O=r["O"].reshape(sh.B, nG, P, G, d),
+                idx=r["idx"].reshape(sh.B, nG, P, K),
+                shat_sel=r["shat_sel"].reshape(sh.B, nG, P, G, K),
+                gap=r["gap"].reshape(sh.B, nG, P),
+                akth=r["akth"].reshape(sh.B, nG, P))
+
+
+def bind_at(inp, positions):
+    """Host copies for ``prefill_at`` at ``positions``: the Q / Qs rows at
+    those positions, K, V, Klm and bias whole."""
+    import torch
+    sh = inp["shape"]
+    pos = np.asarray(positions, dtype=np.int64)
+    pt = torch.as_tensor(pos, device=inp["Q"].device)
+    Qsub = inp["Q"].index_select(2, pt)
+    Qssub = inp["Qs"].index_select(2, pt) if inp.get("Qs") is not None \
+        else None
+    return _Bound(Qsub, Qssub, inp["K"], inp["V"], inp["Klm"], inp["bias"],
+                  inp["head_map"], sh.S, sh.W, sh.K, q_rows=len(pos))

@@ -68,7 +68,8 @@ class Shape:
         return replace(self, **kw)
 
 
-# The five workloads of the scope table, numbered as there.
+# The five benchmark workloads (1: small f32 check; 2, 3, 5: prefill at
+# 32K, 128K, 512K; 4: batch-8 decode over 512K caches).
 PREFILL_CONFIGS = {
     1: Shape("f32", 1, 1, 1, 64, 1024, 64, 128, 4, "plain"),
     2: Shape("bf16", 1, 32, 8, 128, 32768, 64, 512, 16, "needles", n_needles=8),

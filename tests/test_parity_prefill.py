@@ -1,8 +1,12 @@
 """GPU parity of hils_fwd_prefill (through the C ABI) against the fp64 oracle.
 
-Small problems are compared on every row; the full-size workloads of the
-scope table on edge + random rows (oracle row by row), in the same launch
-configuration the benchmark times.
+Small problems are compared on every row. The full-size 32K, 128K and 512K
+workloads run in the launch configuration the benchmark times: at 32K every
+row of one kv group and a few thousand rows of all groups are compared with
+the oracle; at 128K and 512K a few thousand rows of all groups (whole
+128-query blocks at the structural edges, plus rows stratified over the
+chunk phase and the length); on every row the structure of idx is checked
+on the device.
 """
 import numpy as np
 import pytest
@@ -105,9 +109,16 @@ def test_full_size_config_sampled(cfg, cuda_device):
     sh = synth.PREFILL_CONFIGS[cfg]
     inp = synth.make_prefill(sh, seed=synth.seed_for(cfg), device=cuda_device)
     O, idx, sel = run_prefill(inp, sel=True)
-    pos = parity.sample_positions(sh, n_random=40, seed=cfg)
+    pos = parity.sample_positions_dense(sh, n_total=2048, seed=cfg)
+    assert len(pos) >= 2048
     stats = parity.check_prefill(inp, O, idx, positions=pos, sel_gpu=sel)
-    assert stats["rows"] >= len(pos) * sh.Hkv
+    assert stats["rows"] == len(pos) * sh.Hkv * sh.B
+    if cfg == 2:
+        # every row of one kv group (its G heads), against the oracle
+        g = 5
+        stats = parity.check_prefill(inp, O, idx, positions=np.arange(sh.N),
+                                     sel_gpu=sel, groups=[g])
+        assert stats["rows"] == sh.N * sh.B
     # every row's idx is ascending, in C_i, -1 padded (all rows, on device)
     i = torch.arange(sh.N, device=cuda_device)
     nc = torch.clamp(torch.div(i - sh.W + 1, sh.S, rounding_mode="floor"),

@@ -3,10 +3,13 @@
 It is meant for callers that cannot allocate device memory when they call
 (memory reserved up front by a serving loop, latency paths that cannot take
 cudaMalloc's implicit synchronisation, hosts that cannot own a workspace).
-This file checks, through the C ABI, that two consecutive calls give the
-same result as hils_fwd_decode (the entry point with a caller workspace),
-under the tolerance the other parity tests use, and that a shape larger than
-the fixed scratch is refused. Kept in its own file, collected last.
+This file checks, through the C ABI, that each of two consecutive calls
+matches the fp64 oracle (idx exact outside near ties, O within the bf16 /
+f32 bound) and gives the same result as hils_fwd_decode (the entry point with
+a caller workspace), and that a shape larger than the fixed scratch is
+refused. One case has more (sequence, kv head) units than scoring blocks fit
+in the scratch, so the scoring grid is cut to what fits and its blocks loop
+over the units. Kept in its own file, collected last.
 """
 import ctypes
 
@@ -33,15 +36,38 @@ def _noalloc(inp, O, idx):
                                               ctypes.c_void_p(s.cuda_stream))
 
 
-@pytest.mark.parametrize("dtype,lens", [
-    ("bf16", [65536, 40000, 700, 1]),
-    ("f32", [8192, 5000, 513, 64]),
-])
-def test_noalloc_matches_workspace_entry_point(dtype, lens, cuda_device):
-    L = max(lens)
-    sh = synth.Shape(dtype, len(lens), 32 if dtype == "bf16" else 8,
-                     8 if dtype == "bf16" else 2, 128 if dtype == "bf16" else 64,
-                     L, 64, 512, 32 if dtype == "bf16" else 8)
+SCRATCH_BYTES = 8 << 20        # the library's fixed scratch per device
+SM_BLOCKS = 8                  # scoring blocks per SM the launch asks for
+
+CASES = {
+    "bf16_g4": (synth.Shape("bf16", 4, 32, 8, 128, 65536, 64, 512, 32),
+                [65536, 40000, 700, 1]),
+    "f32_g4": (synth.Shape("f32", 4, 8, 2, 64, 8192, 64, 512, 8),
+               [8192, 5000, 513, 64]),
+    # 64 (sequence, kv head) units; one scoring block needs (G+1) x 2040
+    # floats (139 KB), so only 59 blocks fit in the scratch
+    "bf16_g16_grid_cut": (synth.Shape("bf16", 8, 128, 8, 64, 131072, 64, 512,
+                                      32),
+                          [131072, 100000, 65536, 30000, 4096, 700, 64, 1]),
+}
+
+
+def _blocks_that_fit(sh):
+    nc_max = max((sh.N - 1 - sh.W + 1) // sh.S, 1)
+    per_block = 4 * (sh.G + 1) * nc_max
+    sel = -(-4 * sh.B * sh.Hq * sh.K // 256) * 256     # sel_score not given
+    return (SCRATCH_BYTES - sel) // per_block
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_noalloc_matches_workspace_entry_point(name, cuda_device):
+    sh, lens = CASES[name]
+    dtype = sh.dtype
+    if name.endswith("grid_cut"):
+        units = sh.B * sh.Hkv
+        assert _blocks_that_fit(sh) < min(units, SM_BLOCKS * torch.cuda.
+                                          get_device_properties(0).
+                                          multi_processor_count)
     inp = synth.make_decode(sh, seed=404, device=cuda_device, cache_len=lens)
     O_ref, idx_ref = hils.fwd_decode(inp["Q"], inp["K"], inp["V"], inp["Klm"],
                                      inp["bias"], inp["cache_len"],
@@ -55,6 +81,7 @@ def test_noalloc_matches_workspace_entry_point(dtype, lens, cuda_device):
         rc = _noalloc(inp, O, idx)
         assert rc == 0, hils.STATUS.get(rc, rc)
         torch.cuda.synchronize()
+        parity.check_decode(inp, O, idx)            # against the oracle
         a = idx.cpu().numpy()
         b = idx_ref.cpu().numpy()
         differ = (a != b).any(-1)

@@ -440,7 +440,7 @@ class RankContext:
 
 # ---------------------------------------------------------------- GPU arm
 def bench_prefill(args, name, dev, stream, flush, ranks, peaks, steps,
-                  with_e2e, rank):
+                  with_e2e, rank, seq_len=0):
     """Time one prefill workload through the C ABI (select then attend, as
     hils_fwd_prefill runs them), L2 flushed before every timed step.
 
@@ -455,6 +455,8 @@ def bench_prefill(args, name, dev, stream, flush, ranks, peaks, steps,
     import synth
     cfg_id = WORKLOADS[name]
     sh = synth.PREFILL_CONFIGS[cfg_id]
+    if seq_len:
+        sh = sh.with_(N=seq_len)
     inp = synth.make_prefill(sh, seed=synth.seed_for(cfg_id) + 17 * rank,
                              device=dev)
     work = prefill_work(sh)
@@ -536,7 +538,7 @@ def bench_prefill(args, name, dev, stream, flush, ranks, peaks, steps,
            "stages_ms": {"select": s_ms, "attend": a_ms},
            "roofline": roof, "gpu_launches": int(launches),
            "clocks": clk.summary(), "union": union_stats(sh, idx),
-           "config": workload_config(sh, name)}
+           "config": workload_config(sh, name + (f"_n{sh.N}" if seq_len else ""))}
 
     if with_e2e:
         # end to end through the C ABI with host buffers (pinned), per step:
@@ -597,6 +599,9 @@ def main():
                     help="skip the other prefill workloads' legs")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode step (prints its object)")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="run the headline workload at this sequence length "
+                         "instead of its own (reduced cases for profilers)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -632,7 +637,8 @@ def main():
         return
 
     head = bench_prefill(args, args.workload, dev, stream, flush, ranks,
-                         peaks, args.steps, not args.no_e2e, rank)
+                         peaks, args.steps, not args.no_e2e, rank,
+                         seq_len=args.seq_len)
     line = {
         "metric": METRIC, "value": head["value"], "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,

@@ -15,11 +15,11 @@
 //                    window mask, running reference max), stored as bf16 over
 //                    the S columns
 //   O  += P V        tcgen05.mma, 128 x d, A = P from TMEM, f32 in TMEM
-// Shared memory holds only Q and a 2-stage K/V ring (~105 KB) and TMEM 256
-// columns, so two CTAs share an SM and hide each other's latencies. A K
-// stage is handed back when its QK product completes and a V stage when its
-// PV product does, so the copy of K runs ahead and two copies of V are in
-// flight behind the PV chain.
+// Shared memory holds only Q and a K/V ring (two stages at S = 64, one at
+// S = 128; at most ~105 KB) and TMEM 256 columns, so two CTAs share an SM
+// and hide each other's latencies. A K stage is handed back when its QK
+// product completes and a V stage when its PV product does, so the copy of
+// K runs ahead of the PV chain.
 // Warp roles: warp 0 TMA producer (K, V), warp 1 MMA issuer (and TMEM
 // owner), warps 2-5 Q loader, softmax and epilogue (warp w reads TMEM lanes
 // 32*(w%4)..+31). Elementwise softmax arithmetic uses packed f32x2 ops.
@@ -38,7 +38,7 @@ using namespace sm100;
 
 constexpr int kThreads = 192;
 constexpr int kRows = 128;
-constexpr int kStages = 2;
+constexpr int kMaxStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;      // lazy O rescale threshold (log2)
 
@@ -62,27 +62,34 @@ __device__ __forceinline__ void acc_bf16x2(float2 &a, uint32_t v) {
         : "+f"(a.x), "+f"(a.y) : "r"(v));
 }
 
+// Two CTAs share an SM in every configuration: TMEM holds O (D columns) and
+// NSB buffers of S / P (S_TOK columns each) within 256 columns, shared
+// memory Q and NST stages each of K and V. With S_TOK = 64 both are double
+// buffered; with S_TOK = 128 one S buffer and one K / V stage fit, and the
+// other CTA on the SM covers the latencies the single buffers expose.
 template <int S_TOK, int D>
 struct AttnLayout {
+    static constexpr int NSB = (D + 2 * S_TOK) <= 256 ? 2 : 1;   // S buffers
+    static constexpr int NST = NSB;                              // K/V stages
     static constexpr uint32_t Q_BYTES = kRows * D * 2;
     static constexpr uint32_t KV_BYTES = S_TOK * D * 2;        // one of K or V
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
-    static constexpr uint32_t OFF_V = OFF_K + kStages * KV_BYTES;
-    static constexpr uint32_t OFF_SMALL = OFF_V + kStages * KV_BYTES;
+    static constexpr uint32_t OFF_V = OFF_K + NST * KV_BYTES;
+    static constexpr uint32_t OFF_SMALL = OFF_V + NST * KV_BYTES;
     static constexpr int TMEM_O = 0;                 // columns [0, D)
-    static constexpr int TMEM_S = D;                 // 2 buffers of S_TOK (S, then P)
-    static constexpr uint32_t TMEM_COLS =
-        (D + 2 * S_TOK) <= 256 ? 256u : 512u;
-    static constexpr int MIN_BLOCKS = (TMEM_COLS <= 256) ? 2 : 1;
+    static constexpr int TMEM_S = D;                 // NSB buffers of S_TOK (S, then P)
+    static constexpr uint32_t TMEM_COLS = 256u;
+    static constexpr int MIN_BLOCKS = 2;
+    static_assert(D + NSB * S_TOK <= 256, "TMEM budget of two CTAs per SM");
 };
 
 struct SmallState {
     uint64_t q_full;
-    uint64_t k_full[kStages];
-    uint64_t v_full[kStages];
-    uint64_t k_empty[kStages];                       // QK of that stage done
-    uint64_t v_empty[kStages];                       // PV of that stage done
+    uint64_t k_full[kMaxStages];
+    uint64_t v_full[kMaxStages];
+    uint64_t k_empty[kMaxStages];                    // QK of that stage done
+    uint64_t v_empty[kMaxStages];                    // PV of that stage done
     uint64_t s_full[2];
     uint64_t p_full[2];
     uint64_t p_empty[2];                             // PV of that buffer done
@@ -100,6 +107,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV,
                  const TcParams p) {
     using L = AttnLayout<S_TOK, D>;
+    constexpr int NSB = L::NSB, NST = L::NST;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     SmallState &st = *reinterpret_cast<SmallState *>(smem + L::OFF_SMALL);
@@ -120,13 +128,13 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
     // ---------------------------------------------------------- prologue
     if (threadIdx.x == 0) {
         mbar_init(&st.q_full, 128);             // the softmax threads load Q
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(&st.k_full[s], 1);
             mbar_init(&st.v_full[s], 1);
             mbar_init(&st.k_empty[s], 1);
             mbar_init(&st.v_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < NSB; ++s) {
             mbar_init(&st.s_full[s], 1);
             mbar_init(&st.p_full[s], 128);
             mbar_init(&st.p_empty[s], 1);
@@ -223,7 +231,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
             // V once the PV product is: K copies run ahead of V copies, and
             // two V copies stay in flight behind the PV chain.
             auto load = [&](int t, bool is_v) {
-                const int s = t % kStages;
+                const int s = t % NST;
                 const int row = (t < U) ? s_union[t] * p.S
                                         : wstart + (t - U) * S_TOK;
                 uint64_t *bar = is_v ? &st.v_full[s] : &st.k_full[s];
@@ -236,30 +244,30 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
             int nk = 0, nv = 0;                          // copies issued
             while (nv < T) {
                 // next K copy whose stage is already free, else the next V copy
-                if (nk < T && nk < nv + kStages &&
-                    (nk < kStages ||
-                     mbar_test(smem_u32(&st.k_empty[nk % kStages]), ((nk / kStages) - 1) & 1))) {
+                if (nk < T && nk < nv + NST &&
+                    (nk < NST ||
+                     mbar_test(smem_u32(&st.k_empty[nk % NST]), ((nk / NST) - 1) & 1))) {
                     load(nk++, false);
                     continue;
                 }
                 if (nv < nk) {
-                    if (nv >= kStages &&
-                        !mbar_wait(&st.v_empty[nv % kStages], ((nv / kStages) - 1) & 1, abort))
+                    if (nv >= NST &&
+                        !mbar_wait(&st.v_empty[nv % NST], ((nv / NST) - 1) & 1, abort))
                         break;
                     load(nv++, true);
                     continue;
                 }
                 // nv == nk: the K copy must go first
-                if (!mbar_wait(&st.k_empty[nk % kStages], ((nk / kStages) - 1) & 1, abort))
+                if (!mbar_wait(&st.k_empty[nk % NST], ((nk / NST) - 1) & 1, abort))
                     break;
                 load(nk++, false);
             }
             // on abort: let the copies already issued land before exiting
             if (*abort) {
-                for (int t = (nk > kStages ? nk - kStages : 0); t < nk; ++t)
-                    mbar_drain(&st.k_full[t % kStages], (t / kStages) & 1);
-                for (int t = (nv > kStages ? nv - kStages : 0); t < nv; ++t)
-                    mbar_drain(&st.v_full[t % kStages], (t / kStages) & 1);
+                for (int t = (nk > NST ? nk - NST : 0); t < nk; ++t)
+                    mbar_drain(&st.k_full[t % NST], (t / NST) & 1);
+                for (int t = (nv > NST ? nv - NST : 0); t < nv; ++t)
+                    mbar_drain(&st.v_full[t % NST], (t / NST) & 1);
             }
         }
     } else if (warp == 1) {
@@ -273,10 +281,10 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
             bool ok = mbar_wait(&st.q_full, 0, abort);
             tc_fence_after();
             auto do_pv = [&](int u) -> bool {
-                const int pb = u & 1;
-                if (!mbar_wait(&st.p_full[pb], (u >> 1) & 1, abort)) return false;
-                const int s = u % kStages;
-                if (!mbar_wait(&st.v_full[s], (u / kStages) & 1, abort)) return false;
+                const int pb = u % NSB;
+                if (!mbar_wait(&st.p_full[pb], (u / NSB) & 1, abort)) return false;
+                const int s = u % NST;
+                if (!mbar_wait(&st.v_full[s], (u / NST) & 1, abort)) return false;
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < S_TOK / 16; ++k) {
@@ -291,11 +299,13 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                 return true;
             };
             for (int t = 0; ok && t < T; ++t) {
-                const int s = t % kStages;
-                const int sb = t & 1;
-                if (!mbar_wait(&st.k_full[s], (t / kStages) & 1, abort)) { ok = false; break; }
-                // S buffer sb is free once PV(t-2), which read its P, is done
-                if (t >= 2 && !mbar_wait(&st.p_empty[sb], ((t - 2) >> 1) & 1, abort)) { ok = false; break; }
+                const int s = t % NST;
+                const int sb = t % NSB;
+                // one S buffer: PV(t-1) reads its P, so it goes first
+                if (NSB == 1 && t >= 1 && !do_pv(t - 1)) { ok = false; break; }
+                if (!mbar_wait(&st.k_full[s], (t / NST) & 1, abort)) { ok = false; break; }
+                // S buffer sb is free once PV(t-NSB), which read its P, is done
+                if (t >= NSB && !mbar_wait(&st.p_empty[sb], ((t / NSB) - 1) & 1, abort)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
@@ -308,7 +318,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                 }
                 mma_commit(&st.s_full[sb]);
                 mma_commit(&st.k_empty[s]);
-                if (t >= 1 && !do_pv(t - 1)) { ok = false; break; }
+                if (NSB > 1 && t >= 1 && !do_pv(t - 1)) { ok = false; break; }
             }
             if (ok && T > 0) do_pv(T - 1);
             // every MMA of this CTA has completed before TMEM is released
@@ -382,17 +392,18 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
         bool ok = true;
 
         for (int t = 0; t < T; ++t) {
-            const int sb = t & 1;
+            const int sb = t % NSB;
             const uint32_t tS = trow + L::TMEM_S + sb * S_TOK;
             // every lane takes the same branch around warp-collective
             // tcgen05.ld / st, so wait outcomes are agreed across the warp
-            if (!__all_sync(0xffffffffu, mbar_wait(&st.s_full[sb], (t >> 1) & 1, abort))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(&st.s_full[sb], (t / NSB) & 1, abort))) { ok = false; break; }
             tc_fence_after();
-            uint32_t pk[S_TOK / 2];                      // P, bf16 pairs
             float2 ps[4];                                // sum of the rounded P
 #pragma unroll
             for (int k = 0; k < 4; ++k) ps[k] = make_float2(0.f, 0.f);
-
+            // chunk tiles: does this row's query select the chunk, and s^_c
+            bool sel = false;
+            float sh = 0.f;
             if (t < U) {
                 const int c = s_union[t];
                 int ck = kp < p.K ? myidx[kp * M_] : 0x7fffffff;
@@ -401,13 +412,51 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                     ck = kp < p.K ? myidx[kp * M_] : 0x7fffffff;
                     sh_next = (valid && kp < p.K) ? __ldg(mysel + kp) : 0.f;
                 }
-                const bool sel = valid && kp < p.K && ck == c;
-                float sh = 0.f;
+                sel = valid && kp < p.K && ck == c;
                 if (sel) {
                     sh = sh_next * kLog2e;
                     ++kp;
                     sh_next = (kp < p.K) ? __ldg(mysel + kp) : 0.f;
                 }
+            }
+            const int j0 = wstart + (t - U) * S_TOK;     // window tiles
+            // masks only where a row's window starts or ends in the tile
+            const bool edge = t >= U && (!valid || j0 < w0 || j0 + S_TOK - 1 > i);
+            const bool any_edge = __any_sync(0xffffffffu, edge);
+            // raise the reference max of the rows whose window scores exceed
+            // it by more than 2^8 and rescale their O once PV(t-1) is done
+            // (warp-wide: the TMEM load / store are collective; other rows
+            // use a factor of 1). Returns false if the wait gave up.
+            auto window_rescale = [&](float mx) -> bool {
+                const bool mine = mx > mref + kRescaleLog2;
+                if (__any_sync(0xffffffffu, mine)) {
+                    const float fac = !mine ? 1.f
+                                    : (mref == -INFINITY) ? 0.f : fast_exp2(mref - mx);
+                    if (t >= 1) {
+                        const int u = t - 1;
+                        if (!__all_sync(0xffffffffu, mbar_wait(&st.p_empty[u % NSB], (u / NSB) & 1, abort)))
+                            return false;
+                        tc_fence_after();
+#pragma unroll
+                        for (int c0 = 0; c0 < D; c0 += 16) {
+                            uint32_t ro[16];
+                            tmem_ld16(trow + L::TMEM_O + c0, ro);
+                            tmem_wait_ld();
+#pragma unroll
+                            for (int j = 0; j < 16; ++j)
+                                ro[j] = __float_as_uint(__uint_as_float(ro[j]) * fac);
+                            tmem_st16(trow + L::TMEM_O + c0, ro);
+                        }
+                        tmem_wait_st();
+                    }
+                    if (mine) { l *= fac; mref = mx; }
+                }
+                return true;
+            };
+
+            if constexpr (S_TOK <= 64) {
+            uint32_t pk[S_TOK / 2];                      // P, bf16 pairs
+            if (t < U) {
                 if (__any_sync(0xffffffffu, sel)) {
                     uint32_t rr[S_TOK];
 #pragma unroll
@@ -447,14 +496,11 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                     for (int j = 0; j < S_TOK / 2; ++j) pk[j] = 0u;
                 }
             } else {
-                const int j0 = wstart + (t - U) * S_TOK;
                 uint32_t rr[S_TOK];
 #pragma unroll
                 for (int c0 = 0; c0 < S_TOK; c0 += 32) tmem_ld32(tS + c0, rr + c0);
                 tmem_wait_ld();
-                // masks only where a row's window starts or ends in the tile
-                const bool edge = !valid || j0 < w0 || j0 + S_TOK - 1 > i;
-                if (__any_sync(0xffffffffu, edge)) {
+                if (any_edge) {
 #pragma unroll
                     for (int j = 0; j < S_TOK; ++j) {
                         const int pos = j0 + j;
@@ -462,32 +508,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                         rr[j] = in ? rr[j] : __float_as_uint(-INFINITY);
                     }
                 }
-                float mx = row_max(rr, S_TOK) * sl2;         // log2 units
-                const bool mine = mx > mref + kRescaleLog2;
-                if (__any_sync(0xffffffffu, mine)) {
-                    // raise the reference max of the rows that need it and
-                    // rescale their O once PV(t-1) is done (warp-wide: the
-                    // TMEM load / store are collective; other rows use 1)
-                    const float fac = !mine ? 1.f
-                                    : (mref == -INFINITY) ? 0.f : fast_exp2(mref - mx);
-                    if (t >= 1) {
-                        const int u = t - 1;
-                        if (!__all_sync(0xffffffffu, mbar_wait(&st.p_empty[u & 1], (u >> 1) & 1, abort))) { ok = false; break; }
-                        tc_fence_after();
-#pragma unroll
-                        for (int c0 = 0; c0 < D; c0 += 16) {
-                            uint32_t ro[16];
-                            tmem_ld16(trow + L::TMEM_O + c0, ro);
-                            tmem_wait_ld();
-#pragma unroll
-                            for (int j = 0; j < 16; ++j)
-                                ro[j] = __float_as_uint(__uint_as_float(ro[j]) * fac);
-                            tmem_st16(trow + L::TMEM_O + c0, ro);
-                        }
-                        tmem_wait_st();
-                    }
-                    if (mine) { l *= fac; mref = mx; }
-                }
+                if (!window_rescale(row_max(rr, S_TOK) * sl2)) { ok = false; break; }
                 // rows with nothing in the window yet keep mref = -inf:
                 // their masked scores still give exp2(-inf) = 0
                 const float nm = (mref == -INFINITY) ? 0.f : -mref;
@@ -502,14 +523,155 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
                     acc_bf16x2(ps[j & 3], pk[j]);
                 }
             }
-
             // P -> TMEM over this tile's S columns (bf16 pairs), then the MMA.
+#pragma unroll
+            for (int c0 = 0; c0 < S_TOK / 2; c0 += 32) tmem_st32(tS + c0, pk + c0);
+            } else {
+            // S_TOK = 128: the scores are handled in 64-column halves (two
+            // CTAs per SM leave no room for 128 scores next to their
+            // exponentials). P of tokens [0, 64) goes to columns [0, 32),
+            // of tokens [64, 128) to [32, 64); each store lands on columns
+            // whose f32 scores were already read.
+            uint32_t rr[64];
+            if (t < U) {
+                if (__any_sync(0xffffffffu, sel)) {
+                    tmem_ld32(tS + 0, rr);
+                    tmem_ld32(tS + 32, rr + 32);
+                    tmem_wait_ld();
+                    float mx = row_max(rr, 64);
+                    tmem_ld32(tS + 64, rr);
+                    tmem_ld32(tS + 96, rr + 32);
+                    tmem_wait_ld();
+                    mx = fmaxf(mx, row_max(rr, 64));
+                    const float2 nb = make_float2(-mx * sl2, -mx * sl2);
+                    float2 z2[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) z2[k] = make_float2(0.f, 0.f);
+                    // exponentials of tokens [64, 128): kept in rr (f32 bits)
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        float2 e = f2_fma(make_float2(__uint_as_float(rr[2 * j]),
+                                                      __uint_as_float(rr[2 * j + 1])), sl2v, nb);
+                        e.x = fast_exp2(e.x);
+                        e.y = fast_exp2(e.y);
+                        z2[j & 3] = f2_add(z2[j & 3], e);
+                        rr[2 * j] = __float_as_uint(e.x);
+                        rr[2 * j + 1] = __float_as_uint(e.y);
+                    }
+                    // exponentials of tokens [0, 64): back into their columns
+#pragma unroll
+                    for (int c0 = 0; c0 < 64; c0 += 32) {
+                        uint32_t r0[32];
+                        tmem_ld32(tS + c0, r0);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            float2 e = f2_fma(make_float2(__uint_as_float(r0[2 * j]),
+                                                          __uint_as_float(r0[2 * j + 1])), sl2v, nb);
+                            e.x = fast_exp2(e.x);
+                            e.y = fast_exp2(e.y);
+                            z2[j & 3] = f2_add(z2[j & 3], e);
+                            r0[2 * j] = __float_as_uint(e.x);
+                            r0[2 * j + 1] = __float_as_uint(e.y);
+                        }
+                        tmem_st32(tS + c0, r0);
+                    }
+                    tmem_wait_st();
+                    // intra-chunk softmax scaled by exp(s^_c - M0) / z_c;
+                    // rows that did not select the chunk get zero weights
+                    const float2 zz = f2_add(f2_add(z2[0], z2[1]), f2_add(z2[2], z2[3]));
+                    const float f = sel ? __fdividef(fast_exp2(sh - M0l2), zz.x + zz.y) : 0.f;
+                    const float2 fv = make_float2(f, f);
+#pragma unroll
+                    for (int c0 = 0; c0 < 64; c0 += 32) {
+                        uint32_t r0[32], pk[16];
+                        tmem_ld32(tS + c0, r0);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float2 pv = f2_mul(make_float2(__uint_as_float(r0[2 * j]),
+                                                                 __uint_as_float(r0[2 * j + 1])), fv);
+                            pk[j] = pack_bf16(pv.x, pv.y);
+                            acc_bf16x2(ps[j & 3], pk[j]);
+                        }
+                        tmem_st16(tS + c0 / 2, pk);
+                    }
+                    {
+                        uint32_t pk[32];
+#pragma unroll
+                        for (int j = 0; j < 32; ++j) {
+                            const float2 pv = f2_mul(make_float2(__uint_as_float(rr[2 * j]),
+                                                                 __uint_as_float(rr[2 * j + 1])), fv);
+                            pk[j] = pack_bf16(pv.x, pv.y);
+                            acc_bf16x2(ps[j & 3], pk[j]);
+                        }
+                        tmem_st32(tS + 32, pk);
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 64; ++j) rr[j] = 0u;
+                    tmem_st32(tS + 0, rr);
+                    tmem_st32(tS + 32, rr + 32);
+                }
+            } else {
+                // masked row max over both halves
+                float mx = -INFINITY;
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    tmem_ld32(tS + 64 * hf, rr);
+                    tmem_ld32(tS + 64 * hf + 32, rr + 32);
+                    tmem_wait_ld();
+                    if (any_edge) {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) {
+                            const int pos = j0 + 64 * hf + j;
+                            const bool in = valid && pos >= w0 && pos <= i;
+                            rr[j] = in ? rr[j] : __float_as_uint(-INFINITY);
+                        }
+                    }
+                    mx = fmaxf(mx, row_max(rr, 64));
+                }
+                if (!window_rescale(mx * sl2)) { ok = false; break; }
+                const float nm = (mref == -INFINITY) ? 0.f : -mref;
+                const float2 nmv = make_float2(nm, nm);
+                // half 1 is still in rr: its P goes to columns [32, 64) only
+                // after half 0 (columns [0, 64)) has been read back
+                uint32_t pk[32];
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t r0[64];
+                    const uint32_t *src = rr;
+                    if (hf == 0) {
+                        tmem_ld32(tS + 0, r0);
+                        tmem_ld32(tS + 32, r0 + 32);
+                        tmem_wait_ld();
+                        if (any_edge) {
+#pragma unroll
+                            for (int j = 0; j < 64; ++j) {
+                                const int pos = j0 + j;
+                                const bool in = valid && pos >= w0 && pos <= i;
+                                r0[j] = in ? r0[j] : __float_as_uint(-INFINITY);
+                            }
+                        }
+                        src = r0;
+                    }
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        float2 e = f2_fma(make_float2(__uint_as_float(src[2 * j]),
+                                                      __uint_as_float(src[2 * j + 1])), sl2v, nmv);
+                        e.x = fast_exp2(e.x);
+                        e.y = fast_exp2(e.y);
+                        pk[j] = pack_bf16(e.x, e.y);
+                        acc_bf16x2(ps[j & 3], pk[j]);
+                    }
+                    tmem_st32(tS + 32 * hf, pk);
+                }
+            }
+            }
             // The normaliser l sums the rounded weights the MMA consumes, so
             // the weights applied to V add up to one: in a peaked row the
             // rounding of P then moves O by ~2^-9 w(1-w)|v| instead of
             // ~2^-9 w|v|.
-#pragma unroll
-            for (int c0 = 0; c0 < S_TOK / 2; c0 += 32) tmem_st32(tS + c0, pk + c0);
             {
                 const float2 pt = f2_add(f2_add(ps[0], ps[1]), f2_add(ps[2], ps[3]));
                 l += pt.x + pt.y;
@@ -522,7 +684,7 @@ tc_attend_kernel(const __grid_constant__ CUtensorMap tmK,
         // final: O / l once the last PV is done
         if (ok && T > 0) {
             const int u = T - 1;
-            ok = __all_sync(0xffffffffu, mbar_wait(&st.p_empty[u & 1], (u >> 1) & 1, abort));
+            ok = __all_sync(0xffffffffu, mbar_wait(&st.p_empty[u % NSB], (u / NSB) & 1, abort));
         }
         if (ok) {
             tc_fence_after();
@@ -583,7 +745,8 @@ cudaError_t launch_attend_t(const TcParams &tp, const TcMaps &maps,
 }  // namespace
 
 size_t tc_attend_smem_bytes(const TcParams &tp, int s_tok, int d) {
-    size_t big = (size_t)kRows * d * 2 + 2ull * kStages * s_tok * d * 2;
+    const size_t nst = (d + 2 * s_tok) <= 256 ? 2 : 1;     // AttnLayout::NST
+    size_t big = (size_t)kRows * d * 2 + 2ull * nst * s_tok * d * 2;
     size_t small = sizeof(SmallState) + sizeof(int) * ((size_t)tp.M * tp.K + tp.ucap) +
                    sizeof(uint32_t) * (((size_t)tp.nC + 31) / 32);
     return 1024 + big + ((small + 15) / 16) * 16;

@@ -39,6 +39,10 @@ SMALL = {
     "f32_topk_gt_candidates": (synth.Shape("f32", 1, 2, 1, 64, 512, 32, 64, 64), None),
     "bf16_g4_d128": (synth.Shape("bf16", 2, 8, 2, 128, 3000, 64, 256, 8), None),
     "bf16_d64_S128": (synth.Shape("bf16", 1, 8, 2, 64, 2500, 128, 300, 6), None),
+    "bf16_d128_S128_ragged": (synth.Shape("bf16", 2, 8, 2, 128, 5001, 128, 700, 12,
+                                          "needles", n_needles=3), None),
+    "bf16_d128_S128_k32": (synth.Shape("bf16", 1, 8, 2, 128, 9000, 128, 2048, 32,
+                                       "temperature"), None),
     "bf16_qcal": (synth.Shape("bf16", 1, 8, 2, 128, 2048, 64, 200, 4, "qcal"), None),
     "bf16_temperature": (synth.Shape("bf16", 1, 8, 2, 128, 4096, 64, 512, 16, "temperature"), None),
     "bf16_needles": (synth.Shape("bf16", 1, 8, 2, 128, 4096, 64, 512, 16, "needles", n_needles=4), None),

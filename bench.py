@@ -292,7 +292,7 @@ def profiled_traffic(kernels, workload):
         return None
     total = 0
     for k in kernels:
-        ent = tab.get(k)
+        ent = tab.get(f"{k}@{workload}") or tab.get(k)
         if not ent or ent.get("workload") != workload:
             return None
         try:

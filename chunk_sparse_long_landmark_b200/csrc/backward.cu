@@ -383,13 +383,17 @@ bwd_keys_kernel(const BwdParams p) {
     constexpr int NT = S_TOK * kKeySplit;
     extern __shared__ __align__(16) uint8_t smem_raw[];
     KeySmem<D, GM> &sm = *reinterpret_cast<KeySmem<D, GM> *>(smem_raw);
-    const int nchunks = (p.N + S_TOK - 1) / S_TOK;
-    const int c = blockIdx.x % nchunks;
-    const int g = (blockIdx.x / nchunks) % p.Hkv;
-    const int b = blockIdx.x / (nchunks * p.Hkv);
+    // one CTA per block of S_TOK tokens; a chunk of p.S = m * S_TOK tokens
+    // spans m blocks, and only its first block sums dk' and db'
+    const int nblocks = (p.N + S_TOK - 1) / S_TOK;
+    const int blk = blockIdx.x % nblocks;
+    const int g = (blockIdx.x / nblocks) % p.Hkv;
+    const int b = blockIdx.x / (nblocks * p.Hkv);
+    const int c = blk / (p.S / S_TOK);           // the chunk holding the block
+    const bool first_blk = blk % (p.S / S_TOK) == 0;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int jl = tid / kKeySplit, qd = tid % kKeySplit;
-    const int64_t j = (int64_t)c * S_TOK + jl;   // this thread's token
+    const int64_t j = (int64_t)blk * S_TOK + jl; // this thread's token
     const bool jok = j < p.N;
     const int G = p.G;
     const float isd = p.inv_sqrt_d;
@@ -411,6 +415,7 @@ bwd_keys_kernel(const BwdParams p) {
     const T *Qsp = reinterpret_cast<const T *>(p.Qs ? p.Qs : p.Q);
     const T *dOp = reinterpret_cast<const T *>(p.dO);
     const bool is_lm = c < p.nC;                 // a complete chunk: selectable
+    const bool own_lm = is_lm && first_blk;      // this CTA writes dk'_c, db'_c
 
     // process the (row, head) pairs of rows list_i[0..nlist) in batches
     auto run_rows = [&](int role) {
@@ -442,7 +447,7 @@ bwd_keys_kernel(const BwdParams p) {
                         sm.a1[e] = p.rowstat[rq * 2 + 1];
                         int64_t w0, nc;
                         bwd_bounds(ri, p.S, p.W, &w0, &nc);
-                        const int64_t base = (int64_t)c * S_TOK;
+                        const int64_t base = (int64_t)blk * S_TOK;
                         sm.lo[e] = (int)max((int64_t)0, w0 - base);
                         sm.hi[e] = (int)min((int64_t)S_TOK - 1, (int64_t)ri - base);
                     }
@@ -497,7 +502,7 @@ bwd_keys_kernel(const BwdParams p) {
                     adk[4 * r + 3] = fmaf(dsj, a.w, adk[4 * r + 3]);
                 }
             }
-            if (role == 0) {                     // k' and b' of the chunk
+            if (role == 0 && own_lm) {           // k' and b' of the chunk
                 for (int k = tid; k < D; k += NT) {
                     float a = sm.dklm[k];
                     for (int e = 0; e < ne; ++e) a = fmaf(sm.dsh[e], sm.qs[e][k / DQ][k % DQ], a);
@@ -547,9 +552,10 @@ bwd_keys_kernel(const BwdParams p) {
             if (sm.nlist > 0) run_rows(0);
         }
     }
-    // rows whose window covers part of the chunk: i in [cS, ...] with w0 <= cS + S - 1
+    // rows whose window covers part of the block: i in [base, ...] with
+    // w0 <= base + S_TOK - 1
     {
-        const int64_t base = (int64_t)c * S_TOK;
+        const int64_t base = (int64_t)blk * S_TOK;
         for (int64_t r0 = base; r0 < p.N; r0 += 1024) {
             __syncthreads();
             if (tid == 0) {
@@ -581,7 +587,7 @@ bwd_keys_kernel(const BwdParams p) {
         }
     }
     __syncthreads();
-    if (is_lm) {
+    if (own_lm) {
         for (int k = tid; k < D; k += NT) p.dKlm[(bg * p.nC + c) * D + k] = sm.dklm[k] * isd;
         if (tid == 0) p.dbias[bg * p.nC + c] = sm.dbias;
     }
@@ -641,7 +647,8 @@ hils_status bwd_problem(const hils_backward_args *a, BwdParams *p, bool need_ptr
     if (a->Hq % a->Hkv) return HILS_ERR_INVALID_ARG;
     if (a->K > HILS_MAX_TOPK || a->Hq > kMaxHeads) return HILS_ERR_UNSUPPORTED;
     const int G = a->Hq / a->Hkv;
-    if (G > 8 || !(a->d == 64 || a->d == 128) || a->S != 64) return HILS_ERR_UNSUPPORTED;
+    if (G > 8 || !(a->d == 64 || a->d == 128) || !(a->S == 64 || a->S == 128))
+        return HILS_ERR_UNSUPPORTED;
     if ((int64_t)a->B * a->Hq * a->N * a->d >= (1ll << 40)) return HILS_ERR_UNSUPPORTED;
     int count[kMaxHeads];
     for (int g = 0; g < a->Hkv; ++g) count[g] = 0;

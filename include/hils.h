@@ -287,7 +287,7 @@ hils_status hils_fwd_decode_multi(const hils_decode_multi_args *args, void *stre
  *   workspace >= hils_bwd_prefill_workspace_size (per (row, head) and
  *   (row, head, selected chunk) softmax statistics).
  * Deterministic: no floating-point atomics; every output element is summed
- * by one thread in a fixed order. Supported: d in {64,128}, S = 64,
+ * by one thread in a fixed order. Supported: d in {64,128}, S in {64,128},
  * G = Hq/Hkv <= 8; other shapes return HILS_ERR_UNSUPPORTED. Two kernel
  * launches on `stream`.
  */

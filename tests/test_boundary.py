@@ -289,7 +289,7 @@ def test_backward_validation(L):
     assert L.hils_bwd_prefill_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
     assert n.value == 4 * (1 * 8 * 1024 * 2 + 1 * 8 * 1024 * 8 * 3)
     fake = 1 << 40
-    for kw, code in [(dict(S=128), 2), (dict(d=96), 2), (dict(K=65), 2),
+    for kw, code in [(dict(S=32), 2), (dict(d=96), 2), (dict(K=65), 2),
                      (dict(dQ=None), 1), (dict(Qs=fake), 1),
                      (dict(workspace_bytes=16), 4), (dict(dK=fake + 8), 3),
                      (dict(Hkv=3), 1), (dict(dtype=5), 1)]:

@@ -51,6 +51,11 @@ CASES = {
     "f32_qcal": synth.Shape("f32", 1, 2, 1, 128, 768, 64, 128, 3, "qcal"),
     "bf16_needles": synth.Shape("bf16", 1, 4, 1, 128, 2048, 64, 256, 8,
                                 "needles", n_needles=3),
+    # 128-token chunks: the key side works in 64-token blocks, two per chunk
+    "bf16_S128_g4_d128_ragged": synth.Shape("bf16", 1, 8, 2, 128, 2500, 128,
+                                            300, 6),
+    "f32_S128_qcal_d64": synth.Shape("f32", 1, 4, 1, 64, 1300, 128, 200, 4,
+                                     "qcal"),
 }
 
 

@@ -6,10 +6,12 @@
 //
 // The step reads every candidate landmark key once (the O(N/S) routing
 // scan) and the selected chunks + window of the caches once:
-//   dec_score   split over chunk ranges: 64-chunk landmark tiles by TMA,
-//               s^ for the G heads of the group (mma.sync m16n8k16 used as a
-//               dot-product engine: 16 chunks x 8 head slots x 16 dims),
-//               raw s^ -> workspace, per-split (max, sum-exp) per head.
+//   dec_score   an equal run of the (b, kv head, 64-chunk tile) space per
+//               CTA, three CTAs per SM: landmark tiles (and their b') by
+//               TMA, s^ for the G heads of the group (mma.sync m16n8k16 used
+//               as a dot-product engine: 16 chunks x 8 head slots x 16
+//               dims), raw s^ -> workspace, per-segment (max, sum-exp) per
+//               head.
 //   dec_select  one CTA per (b, kv head): merge the log-sum-exp partials,
 //               group score a_c = max_h (s^_hc - LSE_h); a provable lower
 //               bound on the K-th best score (from each warp's two best)
@@ -46,7 +48,11 @@ using namespace sm100;
 
 constexpr int kScoreWarps = 4;
 constexpr int kTileChunks = 64;                 // chunks per landmark tile
-constexpr int kScoreStages = 4;
+constexpr int kMaxScanStages = 16;              // landmark tiles in flight per CTA
+// Scan CTAs per SM: three share the SM's 160 KB of landmark stages (the
+// per-tile work of one CTA is latency-bound; measured: one CTA per SM with
+// ten stages 118.8 us per decode step, two 86.0, three 75.8, four 75.8)
+constexpr int kScanCtasPerSm = 3;
 constexpr int kSelThreads = 1024;
 constexpr int kAttThreads = 128;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -69,8 +75,10 @@ struct DecParams {
     int B, Hq, Hkv, G, d, S, W, K, Lmax, nC;
     int T;              // query tokens per sequence (1: plain decode)
     int ncs;            // chunk stride of ws_s (max candidates of any row)
-    int nsplit;         // landmark splits per (b, g)
-    int cps;            // chunks per split (multiple of kTileChunks)
+    int nsplit;         // scan segments per (b, g), at most
+    int scan_tpu;       // landmark tiles per (b, g)
+    int scan_per;       // landmark tiles per scan CTA
+    int scan_stages;    // tiles in flight per scan CTA
     int ntile;          // attention tiles per (b, g): K + window tiles
     int att_per;        // attention tiles per CTA
     float inv_sqrt_d;
@@ -106,6 +114,16 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map,
         : "memory");
 }
 
+// Contiguous global -> shared copy of `bytes` (a multiple of 16, both
+// addresses 16-byte aligned), completing on `bar`.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes,
+                                          uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(smem_u32(dst)), "l"((uint64_t)src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // Byte offset of 16-byte unit u of row r in a TMA 128B-swizzled tile whose
 // rows are 128 bytes (one 64-column half of a d=128 row).
 __device__ __forceinline__ uint32_t swz(int r, int u) {
@@ -124,7 +142,14 @@ __device__ __forceinline__ bool tok_ok(const DecParams &p, int b, int tok,
 }
 
 // --------------------------------------------------------------- dec_score
-// NG column groups of 8: column n = token * G + head slot (n < T*G <= 8*NG).
+// The landmark scan, balanced over the SMs: a fixed number of CTAs per SM,
+// each streaming an equal run of the flattened (unit, tile) space, unit u =
+// (b, kv head),
+// tile = kTileChunks landmark rows of that unit. A run crosses unit
+// boundaries; each stretch of one unit inside a run is a segment, which
+// emits its own (max, sum-exp) partials: segment s of unit u is the one of
+// CTA firstcta(u) + s. NG column groups of 8: column n = token * G + head
+// slot (n < T*G <= 8*NG).
 template <int D, int NG>
 __global__ void __launch_bounds__(kScoreWarps * 32)
 dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
@@ -132,137 +157,214 @@ dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
     constexpr uint32_t STAGE = kTileChunks * D * 2;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    __shared__ uint64_t full[kScoreStages];
+    __shared__ uint64_t full[kMaxScanStages];
     __shared__ float red_m[kScoreWarps][8 * NG], red_s[kScoreWarps][8 * NG];
+    __shared__ __align__(16) float bias_st[kMaxScanStages][kTileChunks];
 
-    const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gi = lane >> 2, t = lane & 3;
     const int G = p.G, T = p.T, ncol = T * G;
-    const int bg = b * p.Hkv + g;
-    if (split == 0 && threadIdx.x < T)           // tickets of dec_attend
-        p.ws_cnt[((int64_t)b * T + threadIdx.x) * p.Hkv + g] = 0;
-    int64_t i, w0, nc;
-    const bool ok = tok_ok(p, b, T - 1, &i, &w0, &nc);   // the last token's nc is the largest
-    if (!ok) {
-        if (split == 0 && threadIdx.x == 0) report(p.status, HILS_ERR_DEVICE_BAD_LENGTH);
-        return;
-    }
-    const int c_begin = split * p.cps;
-    const int c_end = (int)min((int64_t)c_begin + p.cps, nc);
-    const int ntiles = c_end > c_begin ? (c_end - c_begin + kTileChunks - 1) / kTileChunks : 0;
-
-    // scoring queries as the B operand: column n = (token, head slot), rows = dims
+    const int ns = p.scan_stages;
+    // b' comes with its tile (one bulk copy into the stage) when every row
+    // of it starts on a 16-byte boundary; otherwise lanes load it a tile
+    // ahead
+    const bool bias_bulk = (p.nC % 4 == 0) && (((uintptr_t)p.bias & 15u) == 0);
+    const int64_t total = (int64_t)p.B * p.Hkv * p.scan_tpu;
+    const int64_t gt0 = (int64_t)blockIdx.x * p.scan_per;
+    const int64_t gt1 = min(gt0 + p.scan_per, total);
+    const int ntiles = gt1 > gt0 ? (int)(gt1 - gt0) : 0;
     const void *qb = p.Qs ? p.Qs : p.Q;
-    uint32_t bq[NG][D / 16][2];
-#pragma unroll
-    for (int ng = 0; ng < NG; ++ng) {
-        const int n = ng * 8 + gi;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-            bq[ng][ks][0] = bq[ng][ks][1] = 0u;
-            if (n < ncol) {
-                const int h = p.group_heads[g * G + n % G];
-                const uint32_t *q = reinterpret_cast<const uint32_t *>(
-                    reinterpret_cast<const __nv_bfloat16 *>(qb) +
-                    (((int64_t)b * T + n / G) * p.Hq + h) * D);
-                bq[ng][ks][0] = q[(ks * 16 + 2 * t) >> 1];
-                bq[ng][ks][1] = q[(ks * 16 + 8 + 2 * t) >> 1];
-            }
-        }
-    }
-    // candidates of this lane's output columns 8 ng + 2t + k (token of the
-    // column): a token before the last may have fewer
-    int nc_col[NG][2];
-#pragma unroll
-    for (int ng = 0; ng < NG; ++ng)
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            const int n = ng * 8 + 2 * t + k;
-            int64_t ii, ww, nn = 0;
-            if (n < ncol) tok_ok(p, b, n / G, &ii, &ww, &nn);
-            nc_col[ng][k] = (int)nn;
-        }
+    const float sl2 = p.inv_sqrt_d * kLog2e;
+    volatile int dummy_abort = 0;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kScoreStages; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < ns; ++s) mbar_init(&full[s], 1);
         fence_barrier_init();
     }
     __syncthreads();
-    const int64_t row0 = (int64_t)bg * p.nC + c_begin;
-    if (threadIdx.x == 0) {
-        for (int tt = 0; tt < min(ntiles, kScoreStages); ++tt) {
-            mbar_expect_tx(&full[tt], STAGE);
-            for (int hf = 0; hf < HALVES; ++hf)
-                tma_load_2d(smem + tt * STAGE + hf * (kTileChunks * 128), &tmL,
-                            &full[tt], hf * 64, (int)(row0 + tt * kTileChunks));
-        }
-    }
-    // per lane: columns 8 ng + 2t, +1 (when < T*G); running max / sum, log2 units
+    // TMA row of tile k of this run: landmark row u * nC + tile * kTileChunks
+    // of the flattened [B*Hkv*nC, d] map (rows past the unit's candidates
+    // are read and masked). Thread 0 issues the tiles in order; its cursor
+    // (iu, itl) walks the (unit, tile) space without divisions.
+    int iu = (int)(gt0 / p.scan_tpu), itl = (int)(gt0 % p.scan_tpu);
+    auto issue = [&](int k) {
+        const int64_t u = iu, tl = itl;
+        if (++itl == p.scan_tpu) { itl = 0; ++iu; }
+        const int s = k % ns;
+        // b' of the tile's chunks inside [0, nC): a multiple of 4 floats
+        const int nb = bias_bulk ? (int)min((int64_t)kTileChunks, p.nC - tl * kTileChunks) : 0;
+        mbar_expect_tx(&full[s], STAGE + (nb > 0 ? 4u * nb : 0u));
+        for (int hf = 0; hf < HALVES; ++hf)
+            tma_load_2d(smem + s * STAGE + hf * (kTileChunks * 128), &tmL, &full[s],
+                        hf * 64, (int)(u * p.nC + tl * kTileChunks));
+        if (nb > 0)
+            bulk_load(&bias_st[s][0], p.bias + u * p.nC + tl * kTileChunks, 4u * nb, &full[s]);
+    };
+    if (threadIdx.x == 0)
+        for (int k = 0; k < min(ntiles, ns); ++k) issue(k);
+
+    // state of the current unit
+    int cur = -1, b = 0, g = 0, nc_last = 0;
+    uint32_t bq[NG][D / 16][2];
+    int nc_col[NG][2];
     float mx[NG][2], sm[NG][2];
+    // the partials of the unit's segment held by this CTA
+    auto finalize = [&](int u) {
 #pragma unroll
-    for (int ng = 0; ng < NG; ++ng)
-        mx[ng][0] = mx[ng][1] = -INFINITY, sm[ng][0] = sm[ng][1] = 0.f;
-    const float sl2 = p.inv_sqrt_d * kLog2e;
-    const float *bias = p.bias + (int64_t)bg * p.nC;
-    // s^ of column n = (token, head slot) at ((bg * T + token) * G + slot) * ncs
-    float *outs = p.ws_s + (int64_t)bg * T * G * p.ncs;
-    volatile int dummy_abort = 0;
-    // bias of the lane's 2 chunks of the next tile, loaded a tile ahead
-    auto load_bias = [&](int tt, float *bv) {
+        for (int ng = 0; ng < NG; ++ng)
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                for (int o = 4; o < 32; o <<= 1) {
+                    const float om = __shfl_xor_sync(0xffffffffu, mx[ng][k], o);
+                    const float os = __shfl_xor_sync(0xffffffffu, sm[ng][k], o);
+                    const float mn = fmaxf(mx[ng][k], om);
+                    sm[ng][k] = (mn == -INFINITY) ? 0.f
+                                : sm[ng][k] * fast_exp2(mx[ng][k] - mn) + os * fast_exp2(om - mn);
+                    mx[ng][k] = mn;
+                }
+                if (gi == 0) {
+                    red_m[warp][ng * 8 + 2 * t + k] = mx[ng][k];
+                    red_s[warp][ng * 8 + 2 * t + k] = sm[ng][k];
+                }
+            }
+        __syncthreads();
+        if (threadIdx.x < ncol) {
+            const int n = threadIdx.x;
+            float m = -INFINITY, s2 = 0.f;
+            for (int w = 0; w < kScoreWarps; ++w) {
+                const float om = red_m[w][n], os = red_s[w][n];
+                const float mn = fmaxf(m, om);
+                s2 = (mn == -INFINITY) ? 0.f : s2 * fast_exp2(m - mn) + os * fast_exp2(om - mn);
+                m = mn;
+            }
+            const int seg = (int)blockIdx.x - (int)(((int64_t)u * p.scan_tpu) / p.scan_per);
+            // partials of (b, g, token) at ((u * T + token) * nsplit + seg) * G + slot
+            float *pp = p.ws_p + ((((int64_t)u * T + n / G) * p.nsplit + seg) * G + n % G) * 2;
+            pp[0] = m;          // log2 units
+            pp[1] = s2;
+        }
+        __syncthreads();                         // red_m / red_s free again
+    };
+    auto setup = [&](int u, bool first_tile) {
+        b = u / p.Hkv;
+        g = u - b * p.Hkv;
+        if (first_tile && threadIdx.x < T)       // tickets of dec_attend
+            p.ws_cnt[((int64_t)b * T + threadIdx.x) * p.Hkv + g] = 0;
+        int64_t i, w0, nc = 0;
+        if (!tok_ok(p, b, T - 1, &i, &w0, &nc)) {
+            nc = 0;                              // reported once, scanned as empty
+            if (first_tile && threadIdx.x == 0) report(p.status, HILS_ERR_DEVICE_BAD_LENGTH);
+        }
+        nc_last = (int)nc;                       // the last token's nc is the largest
+        // scoring queries as the B operand: column n = (token, head slot), rows = dims
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng) {
+            const int n = ng * 8 + gi;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                bq[ng][ks][0] = bq[ng][ks][1] = 0u;
+                if (n < ncol) {
+                    const int h = p.group_heads[g * G + n % G];
+                    const uint32_t *q = reinterpret_cast<const uint32_t *>(
+                        reinterpret_cast<const __nv_bfloat16 *>(qb) +
+                        (((int64_t)b * T + n / G) * p.Hq + h) * D);
+                    bq[ng][ks][0] = q[(ks * 16 + 2 * t) >> 1];
+                    bq[ng][ks][1] = q[(ks * 16 + 8 + 2 * t) >> 1];
+                }
+            }
+        }
+        // candidates of this lane's output columns 8 ng + 2t + k (token of
+        // the column): a token before the last may have fewer
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng)
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int n = ng * 8 + 2 * t + k;
+                int64_t ii, ww, nn = 0;
+                if (n < ncol && nc_last > 0) tok_ok(p, b, n / G, &ii, &ww, &nn);
+                nc_col[ng][k] = (int)nn;
+                mx[ng][k] = -INFINITY;
+                sm[ng][k] = 0.f;
+            }
+    };
+    // bias of the lane's 2 chunks of tile k, loaded a tile ahead
+    auto load_bias = [&](int k, int u, int tl, float *bv) {
+        bv[0] = bv[1] = 0.f;
+        if (bias_bulk || k >= ntiles) return;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
-            const int c = c_begin + tt * kTileChunks + warp * 16 + gi + q * 8;
-            bv[q] = (tt < ntiles && c < c_end) ? __ldg(bias + c) : 0.f;
+            const int c = (int)tl * kTileChunks + warp * 16 + gi + q * 8;
+            if (c < p.nC) bv[q] = __ldg(p.bias + u * p.nC + c);
         }
     };
+    // consumer cursor over (unit, tile), and the next tile's
+    int u = (int)(gt0 / p.scan_tpu), tl = (int)(gt0 % p.scan_tpu);
+    int un = u, tn = tl + 1;
+    if (tn == p.scan_tpu) { tn = 0; ++un; }
     float bnext[2];
-    load_bias(0, bnext);
-    for (int tt = 0; tt < ntiles; ++tt) {
-        const int s = tt % kScoreStages;
-        const float bcur[2] = {bnext[0], bnext[1]};
-        load_bias(tt + 1, bnext);
-        mbar_wait(&full[s], (tt / kScoreStages) & 1, &dummy_abort);
-        float acc[NG][4];
+    load_bias(0, u, tl, bnext);
+    for (int k = 0; k < ntiles; ++k) {
+        if (k > 0) {
+            u = un; tl = tn;
+            if (++tn == p.scan_tpu) { tn = 0; ++un; }
+        }
+        if (u != cur) {                          // uniform over the CTA
+            if (cur >= 0) finalize(cur);
+            setup(u, tl == 0);
+            cur = u;
+        }
+        const int s = k % ns;
+        float bcur[2] = {bnext[0], bnext[1]};
+        load_bias(k + 1, un, tn, bnext);
+        mbar_wait(&full[s], (k / ns) & 1, &dummy_abort);
+        if (bias_bulk) {
+            bcur[0] = bias_st[s][warp * 16 + gi];
+            bcur[1] = bias_st[s][warp * 16 + gi + 8];
+        }
+        // two independent accumulator chains (even / odd k-steps) halve the
+        // dependent MMA latency of a tile
+        float acc[NG][4], acc2[NG][4];
 #pragma unroll
-        for (int ng = 0; ng < NG; ++ng) acc[ng][0] = acc[ng][1] = acc[ng][2] = acc[ng][3] = 0.f;
+        for (int ng = 0; ng < NG; ++ng)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[ng][q] = acc2[ng][q] = 0.f;
         const uint32_t base = smem_u32(smem + s * STAGE);
         const int r = warp * 16 + (lane & 15);
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-            const int hf = ks / 4, u = (ks % 4) * 2 + (lane >> 4);
+            const int hf = ks / 4, uu = (ks % 4) * 2 + (lane >> 4);
             uint32_t a[4];
-            ldsm_x4(base + hf * (kTileChunks * 128) + swz(r, u), a);
+            ldsm_x4(base + hf * (kTileChunks * 128) + swz(r, uu), a);
 #pragma unroll
             for (int ng = 0; ng < NG; ++ng)
-                if (ng * 8 < ncol) mma_bf16(acc[ng], a, bq[ng][ks][0], bq[ng][ks][1]);
+                if (ng * 8 < ncol) mma_bf16((ks & 1) ? acc2[ng] : acc[ng], a, bq[ng][ks][0], bq[ng][ks][1]);
         }
+#pragma unroll
+        for (int ng = 0; ng < NG; ++ng)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[ng][q] += acc2[ng][q];
         __syncthreads();                         // stage s fully read
-        if (threadIdx.x == 0 && tt + kScoreStages < ntiles) {
-            const int tn = tt + kScoreStages;
-            mbar_expect_tx(&full[s], STAGE);
-            for (int hf = 0; hf < HALVES; ++hf)
-                tma_load_2d(smem + s * STAGE + hf * (kTileChunks * 128), &tmL,
-                            &full[s], hf * 64, (int)(row0 + tn * kTileChunks));
-        }
+        if (threadIdx.x == 0 && k + ns < ntiles) issue(k + ns);
+        // s^ of column n = (token, head slot) at ((u * T + token) * G + slot) * ncs
+        float *outs = p.ws_s + (int64_t)u * T * G * p.ncs;
         // acc[ng]: chunks (gi, gi+8) of this warp's 16, columns 8 ng + (2t, 2t+1)
 #pragma unroll
         for (int ng = 0; ng < NG; ++ng)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int n = ng * 8 + 2 * t + (q & 1);
-                const int k = q & 1;
-                const int c = c_begin + tt * kTileChunks + warp * 16 + gi + (q >> 1) * 8;
-                if (n < ncol && c < c_end) {
+                const int kk = q & 1;
+                const int c = tl * kTileChunks + warp * 16 + gi + (q >> 1) * 8;
+                if (n < ncol && c < nc_last) {
                     const float shat = fmaf(acc[ng][q], p.inv_sqrt_d, bcur[q >> 1]);
                     outs[(int64_t)n * p.ncs + c] = shat;
-                    if (c < nc_col[ng][k]) {
+                    if (c < nc_col[ng][kk]) {
                         const float x = shat * kLog2e;
-                        if (x > mx[ng][k]) {
-                            sm[ng][k] = sm[ng][k] * fast_exp2(mx[ng][k] - x) + 1.f;
-                            mx[ng][k] = x;
+                        if (x > mx[ng][kk]) {
+                            sm[ng][kk] = sm[ng][kk] * fast_exp2(mx[ng][kk] - x) + 1.f;
+                            mx[ng][kk] = x;
                         } else {
-                            sm[ng][k] += fast_exp2(x - mx[ng][k]);
+                            sm[ng][kk] += fast_exp2(x - mx[ng][kk]);
                         }
                     }
                 }
@@ -273,45 +375,13 @@ dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
     if (dummy_abort) {                           // a tile never arrived
         if (threadIdx.x == 0) {
             report(p.status, HILS_ERR_DEVICE_TIMEOUT);
-            for (int tt = max(0, ntiles - kScoreStages); tt < ntiles; ++tt)
-                mbar_drain(&full[tt % kScoreStages], (tt / kScoreStages) & 1);
+            for (int k = max(0, ntiles - ns); k < ntiles; ++k)
+                mbar_drain(&full[k % ns], (k / ns) & 1);
         }
         __syncthreads();
         return;
     }
-    // reduce (max, sum) over the 8 chunk lanes (gi) then over warps
-#pragma unroll
-    for (int ng = 0; ng < NG; ++ng)
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-            for (int o = 4; o < 32; o <<= 1) {
-                const float om = __shfl_xor_sync(0xffffffffu, mx[ng][k], o);
-                const float os = __shfl_xor_sync(0xffffffffu, sm[ng][k], o);
-                const float mn = fmaxf(mx[ng][k], om);
-                sm[ng][k] = (mn == -INFINITY) ? 0.f
-                            : sm[ng][k] * fast_exp2(mx[ng][k] - mn) + os * fast_exp2(om - mn);
-                mx[ng][k] = mn;
-            }
-            if (gi == 0) {
-                red_m[warp][ng * 8 + 2 * t + k] = mx[ng][k];
-                red_s[warp][ng * 8 + 2 * t + k] = sm[ng][k];
-            }
-        }
-    __syncthreads();
-    if (threadIdx.x < ncol) {
-        const int n = threadIdx.x;
-        float m = -INFINITY, s2 = 0.f;
-        for (int w = 0; w < kScoreWarps; ++w) {
-            const float om = red_m[w][n], os = red_s[w][n];
-            const float mn = fmaxf(m, om);
-            s2 = (mn == -INFINITY) ? 0.f : s2 * fast_exp2(m - mn) + os * fast_exp2(om - mn);
-            m = mn;
-        }
-        // partials of (b, g, token) at ((bg * T + token) * nsplit + split) * G + slot
-        float *pp = p.ws_p + ((((int64_t)bg * T + n / G) * p.nsplit + split) * G + n % G) * 2;
-        pp[0] = m;          // log2 units
-        pp[1] = s2;
-    }
+    if (cur >= 0) finalize(cur);
 }
 
 // -------------------------------------------------------------- dec_select
@@ -443,7 +513,9 @@ dec_select_kernel(const DecParams p) {
 
     // merge the split partials: all loaded at once into shared memory, then
     // folded in split order by one thread per head
-    const int nsp = (nc + p.cps - 1) / p.cps;
+    // the scan segments of this (b, g): CTAs firstcta .. lastcta
+    const int64_t u0 = (int64_t)(b * p.Hkv + g) * p.scan_tpu;
+    const int nsp = (int)((u0 + p.scan_tpu - 1) / p.scan_per - u0 / p.scan_per) + 1;
     const bool staged = nsp * G <= kSelThreads && nsp <= kMaxSplits;
     if (staged && threadIdx.x < nsp * G) {
         const float *pp = p.ws_p + ((int64_t)bgt * p.nsplit * G + threadIdx.x) * 2;
@@ -1043,7 +1115,7 @@ bool map_2d(CUtensorMap *m, const void *base, int d, int64_t rows, int box_rows)
 }
 
 struct DecPlan {
-    int ncs, nsplit, cps, ntile, att_per;
+    int ncs, nsplit, scan_tpu, scan_per, scan_stages, scan_ctas, ntile, att_per;
     size_t off_s, off_p, off_o, off_ml, off_cnt, total;
 };
 
@@ -1053,20 +1125,26 @@ DecPlan dec_plan(const Problem &p) {
     window_bounds((int64_t)p.kv_rows - 1, p.S, p.W, &w0, &ncm);
     // s^ rows padded to a multiple of 4 floats: 16-byte loads in dec_select
     pl.ncs = (int)(((ncm > 0 ? ncm : 1) + 3) & ~(int64_t)3);
-    // splits sized so that about 3 CTAs per SM stream the whole scan
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // one wave: at most 3 resident CTAs per SM (65 KB of stages each); the
+    // the scan: kScanCtasPerSm CTAs per SM, each streaming an equal run of
+    // the (unit, tile) space, 160 KB of landmark tiles in flight per SM; the
     // T tokens of a sequence share its scan
-    const int64_t want = (int64_t)3 * sms;
-    int64_t per_bg = want / ((int64_t)p.B * p.Hkv);
-    if (per_bg < 1) per_bg = 1;
-    int64_t tiles = (pl.ncs + kTileChunks - 1) / kTileChunks;
-    int64_t tps = (tiles + per_bg - 1) / (per_bg > 0 ? per_bg : 1);
-    if (tps < 4) tps = 4;
-    pl.cps = (int)(tps * kTileChunks);
-    pl.nsplit = (pl.ncs + pl.cps - 1) / pl.cps;
+    pl.scan_tpu = (int)((pl.ncs + kTileChunks - 1) / kTileChunks);
+    const int64_t total = (int64_t)p.B * p.Hkv * pl.scan_tpu;
+    const int64_t slots = (int64_t)sms * kScanCtasPerSm;
+    int64_t ctas = total < slots ? total : slots;
+    const int64_t per = (total + ctas - 1) / ctas;
+    pl.scan_per = (int)per;
+    pl.scan_ctas = (int)((total + per - 1) / per);
+    // a unit's tiles lie in at most this many CTA runs
+    pl.nsplit = (pl.scan_tpu + pl.scan_per - 1) / pl.scan_per + 1;
+    {
+        const int stage = kTileChunks * p.d * 2;
+        int ns = (160 * 1024) / kScanCtasPerSm / stage;
+        pl.scan_stages = ns < kMaxScanStages ? ns : kMaxScanStages;
+    }
     pl.ntile = p.K + (p.W + 2 * p.S - 2) / p.S + 1;
     // attention: one wave of CTAs, 2 per SM at S = 64 (measured faster than
     // 3 shorter ones), 1 at S = 128
@@ -1103,7 +1181,8 @@ DecParams dec_params(const Problem &p, void *ws) {
     d.ws_cnt = (int32_t *)(base + pl.off_cnt);
     d.B = p.B; d.Hq = p.Hq; d.Hkv = p.Hkv; d.G = p.G; d.d = p.d; d.S = p.S;
     d.W = p.W; d.K = p.K; d.Lmax = p.kv_rows; d.nC = p.nC; d.T = p.T;
-    d.ncs = pl.ncs; d.nsplit = pl.nsplit; d.cps = pl.cps; d.ntile = pl.ntile;
+    d.ncs = pl.ncs; d.nsplit = pl.nsplit; d.ntile = pl.ntile;
+    d.scan_tpu = pl.scan_tpu; d.scan_per = pl.scan_per; d.scan_stages = pl.scan_stages;
     d.att_per = pl.att_per;
     d.inv_sqrt_d = p.inv_sqrt_d;
     for (int k = 0; k < kMaxHeads; ++k) d.group_heads[k] = p.group_heads[k];
@@ -1161,8 +1240,8 @@ cudaError_t launch_dec_select(Problem &p, void *ws, cudaStream_t st) {
     CUtensorMap tl;
     if (!map_2d(&tl, p.Klm, p.d, (int64_t)p.B * p.Hkv * p.nC, kTileChunks))
         return cudaErrorInvalidValue;
-    const size_t smem = 1024 + (size_t)kScoreStages * kTileChunks * p.d * 2;
-    dim3 grid(d.nsplit, p.Hkv, p.B);
+    const size_t smem = 1024 + (size_t)d.scan_stages * kTileChunks * p.d * 2;
+    dim3 grid((unsigned)dec_plan(p).scan_ctas);
     const int ncol = p.T * p.G;
     cudaError_t e;
     if (p.d == 128) {

@@ -49,7 +49,7 @@ using namespace sm100;
 constexpr int kScoreWarps = 4;
 constexpr int kTileChunks = 64;                 // chunks per landmark tile
 constexpr int kMaxScanStages = 16;              // landmark tiles in flight per CTA
-// Scan CTAs per SM: three share the SM's 160 KB of landmark stages (the
+// Scan CTAs per SM: three share the SM's landmark stages (the
 // per-tile work of one CTA is latency-bound; measured: one CTA per SM with
 // ten stages 118.8 us per decode step, two 86.0, three 75.8, four 75.8)
 constexpr int kScanCtasPerSm = 3;
@@ -347,26 +347,28 @@ dec_score_kernel(const __grid_constant__ CUtensorMap tmL, const DecParams p) {
         if (threadIdx.x == 0 && k + ns < ntiles) issue(k + ns);
         // s^ of column n = (token, head slot) at ((u * T + token) * G + slot) * ncs
         float *outs = p.ws_s + (int64_t)u * T * G * p.ncs;
-        // acc[ng]: chunks (gi, gi+8) of this warp's 16, columns 8 ng + (2t, 2t+1)
+        // acc[ng]: chunks (gi, gi+8) of this warp's 16, columns 8 ng + (2t, 2t+1);
+        // each column's running (max, sum) takes both of its chunks at once
+        const int c_lo = tl * kTileChunks + warp * 16 + gi;
 #pragma unroll
         for (int ng = 0; ng < NG; ++ng)
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int n = ng * 8 + 2 * t + (q & 1);
-                const int kk = q & 1;
-                const int c = tl * kTileChunks + warp * 16 + gi + (q >> 1) * 8;
-                if (n < ncol && c < nc_last) {
-                    const float shat = fmaf(acc[ng][q], p.inv_sqrt_d, bcur[q >> 1]);
-                    outs[(int64_t)n * p.ncs + c] = shat;
-                    if (c < nc_col[ng][kk]) {
-                        const float x = shat * kLog2e;
-                        if (x > mx[ng][kk]) {
-                            sm[ng][kk] = sm[ng][kk] * fast_exp2(mx[ng][kk] - x) + 1.f;
-                            mx[ng][kk] = x;
-                        } else {
-                            sm[ng][kk] += fast_exp2(x - mx[ng][kk]);
-                        }
-                    }
+            for (int kk = 0; kk < 2; ++kk) {
+                const int n = ng * 8 + 2 * t + kk;
+                if (n >= ncol) continue;
+                float x[2];
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int c = c_lo + 8 * h2;
+                    const float shat = fmaf(acc[ng][kk + 2 * h2], p.inv_sqrt_d, bcur[h2]);
+                    if (c < nc_last) outs[(int64_t)n * p.ncs + c] = shat;
+                    x[h2] = (c < nc_col[ng][kk]) ? shat * kLog2e : -INFINITY;
+                }
+                const float mn = fmaxf(mx[ng][kk], fmaxf(x[0], x[1]));
+                if (mn != -INFINITY) {
+                    sm[ng][kk] = sm[ng][kk] * fast_exp2(mx[ng][kk] - mn) +
+                                 fast_exp2(x[0] - mn) + fast_exp2(x[1] - mn);
+                    mx[ng][kk] = mn;
                 }
             }
     }
@@ -1129,7 +1131,7 @@ DecPlan dec_plan(const Problem &p) {
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     // the scan: kScanCtasPerSm CTAs per SM, each streaming an equal run of
-    // the (unit, tile) space, 160 KB of landmark tiles in flight per SM; the
+    // the (unit, tile) space, 192 KB of landmark tiles in flight per SM; the
     // T tokens of a sequence share its scan
     pl.scan_tpu = (int)((pl.ncs + kTileChunks - 1) / kTileChunks);
     const int64_t total = (int64_t)p.B * p.Hkv * pl.scan_tpu;
@@ -1142,7 +1144,7 @@ DecPlan dec_plan(const Problem &p) {
     pl.nsplit = (pl.scan_tpu + pl.scan_per - 1) / pl.scan_per + 1;
     {
         const int stage = kTileChunks * p.d * 2;
-        int ns = (160 * 1024) / kScanCtasPerSm / stage;
+        int ns = (192 * 1024) / kScanCtasPerSm / stage;
         pl.scan_stages = ns < kMaxScanStages ? ns : kMaxScanStages;
     }
     pl.ntile = p.K + (p.W + 2 * p.S - 2) / p.S + 1;

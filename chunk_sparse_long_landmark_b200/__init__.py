@@ -86,7 +86,7 @@ class BackwardArgs(ctypes.Structure):
                 ("bias", _p), ("dO", _p), ("idx", _p), ("dQ", _p),
                 ("dQs", _p), ("dK", _p), ("dV", _p), ("dKlm", _p),
                 ("dbias", _p), ("workspace", _p),
-                ("workspace_bytes", ctypes.c_size_t)]
+                ("workspace_bytes", ctypes.c_size_t), ("status", _p)]
 
 
 class DecodeMultiArgs(ctypes.Structure):

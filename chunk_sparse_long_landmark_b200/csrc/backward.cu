@@ -20,7 +20,7 @@
 //             over the row's tokens (lane per token) give lz_c, L, D, then
 //             p and ds; dq accumulates with lane l owning d/32 dims. Writes
 //             dQ (dQs) and per (row, head) L, D and per (row, head, chunk)
-//             lz, P, Ubar for the key-side kernel.
+//             a = lz_c - s^_c + L, Ubar_c and dsh_c for the key side.
 //   bwd_keys  one CTA per (b, g, chunk of S tokens): the query rows that
 //             selected the chunk (found by scanning idx, ascending) and the
 //             rows whose window covers it, in ascending order; thread
@@ -31,6 +31,7 @@
 #include <stdint.h>
 
 #include "hils_fast.cuh"
+#include "tc_kernels.cuh"
 
 namespace hils {
 namespace {
@@ -44,7 +45,17 @@ struct BwdParams {
     const int32_t *idx;
     float *dQ, *dQs, *dK, *dV, *dKlm, *dbias;
     float *rowstat;     // [B, Hq, N, 2]: L, D
-    float *chunkstat;   // [B, Hq, N, K, 3]: lz, P, Ubar (valid selected entries)
+    // [B, Hq, N, K, 4] for valid selected entries: a = lz_c - s^_c + L (the
+    // chunk's tokens get p_j = exp(s_j - a)), Ubar_c, dsh_c = P_c (Ubar_c - D)
+    float *chunkstat;
+    int *csr_off;       // inverse index (tensor-core key side)
+    int32_t *csr_ent;
+    int2 *units;        // work units of the tensor-core key side
+    int *nunits_blk, *tickets, *n_units;
+    float *partial;
+    int64_t max_units;
+    int32_t *status;
+    bool tc_keys;
     int B, Hq, Hkv, G, N, S, W, K, nC;
     float inv_sqrt_d;
     int16_t group_heads[kMaxHeads];
@@ -343,10 +354,12 @@ bwd_rows_kernel(const BwdParams p) {
             p.rowstat[rq * 2 + 1] = Dr[h];
         }
         for (int n = lane; n < nsel; n += 32) {
-            float *cs = p.chunkstat + (rq * p.K + sm.kpos[n]) * 3;
-            cs[0] = sm.lz[h][n];
-            cs[1] = expf(sm.sh[h][n] - Lr[h]);
-            cs[2] = sm.ub[h][n];
+            // chunk tokens: p_j = exp(s_j - a), a = lz_c - s^_c + L
+            float *cs = p.chunkstat + (rq * p.K + sm.kpos[n]) * 4;
+            const float P = expf(sm.sh[h][n] - Lr[h]);
+            cs[0] = sm.lz[h][n] - sm.sh[h][n] + Lr[h];
+            cs[1] = sm.ub[h][n];
+            cs[2] = P * (sm.ub[h][n] - Dr[h]);
         }
     }
 }
@@ -365,9 +378,9 @@ template <int D, int GM>
 struct KeySmem {
     float q[kKeyBatch][kKeySplit][kSlice<D>], go[kKeyBatch][kKeySplit][kSlice<D>],
           qs[kKeyBatch][kKeySplit][kSlice<D>];
-    // per pair: chunk role (lz, P, Ubar), window role (L, D, -); the row's
-    // token range inside the chunk; dsh = P (Ubar - D) (chunk role)
-    float a0[kKeyBatch], a1[kKeyBatch], a2[kKeyBatch], dsh[kKeyBatch];
+    // per pair: chunk role (a, Ubar), window role (L, D); the row's token
+    // range inside the chunk; dsh = P (Ubar - D) (chunk role)
+    float a0[kKeyBatch], a1[kKeyBatch], dsh[kKeyBatch];
     int lo[kKeyBatch], hi[kKeyBatch];
     float dklm[D];
     float dbias;
@@ -434,12 +447,11 @@ bwd_keys_kernel(const BwdParams p) {
                     if (role == 0) sm.qs[e][k / DQ][k % DQ] = ld_f(Qsp + rq * D + k);
                 }
                 if (lane == 0) {
-                    if (role == 0) {             // lz, P, Ubar and D of the row
-                        const float *cs = p.chunkstat + (rq * p.K + sm.list_k[pr / G]) * 3;
+                    if (role == 0) {             // a, Ubar and dsh of the row
+                        const float *cs = p.chunkstat + (rq * p.K + sm.list_k[pr / G]) * 4;
                         sm.a0[e] = cs[0];
                         sm.a1[e] = cs[1];
-                        sm.a2[e] = cs[2];
-                        sm.dsh[e] = cs[1] * (cs[2] - p.rowstat[rq * 2 + 1]);
+                        sm.dsh[e] = cs[2];
                         sm.lo[e] = 0;
                         sm.hi[e] = S_TOK - 1;
                     } else {                     // L, D and the window's span
@@ -482,8 +494,8 @@ bwd_keys_kernel(const BwdParams p) {
                 float pj = 0.f, dsj = 0.f;
                 if (jok && jl >= sm.lo[e] && jl <= sm.hi[e]) {
                     if (role == 0) {
-                        pj = sm.a1[e] * expf(x - sm.a0[e]);
-                        dsj = pj * (up - sm.a2[e]);
+                        pj = expf(x - sm.a0[e]);
+                        dsj = pj * (up - sm.a1[e]);
                     } else {
                         pj = expf(x - sm.a0[e]);
                         dsj = pj * (up - sm.a1[e]);
@@ -627,6 +639,14 @@ cudaError_t launch_bwd_t(const BwdParams &p, cudaStream_t st) {
 }
 
 template <typename T, int D>
+cudaError_t launch_rows_d(const BwdParams &p, cudaStream_t st) {
+    if (p.G == 1) return launch_rows_t<T, D, 1>(p, st);
+    if (p.G == 2) return launch_rows_t<T, D, 2>(p, st);
+    if (p.G <= 4) return launch_rows_t<T, D, 4>(p, st);
+    return launch_rows_t<T, D, 8>(p, st);
+}
+
+template <typename T, int D>
 cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t st) {
     if (p.G == 1) return launch_bwd_t<T, D, 1>(p, st);
     if (p.G == 2) return launch_bwd_t<T, D, 2>(p, st);
@@ -635,6 +655,18 @@ cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t st) {
 }
 
 bool al16b(const void *q) { return ((uintptr_t)q & 15u) == 0; }
+
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// bf16 problems whose key side runs on the tensor cores
+bool keys_tc_ok(const hils_backward_args *a, int G, int nC) {
+    if (a->dtype != HILS_BF16 || !(a->d == 64 || a->d == 128)) return false;
+    if (!(a->S == 64 || a->S == 128) || G > 8 || a->K > 64) return false;
+    if (a->N >= (1 << 25) || (size_t)nC * sizeof(int) > 200 * 1024) return false;
+    if ((int64_t)a->B * a->Hq * a->N >= (1ll << 31)) return false;
+    if (bwd_keys_tc_smem(a->d, a->Qs != nullptr) > 227 * 1024) return false;
+    return tc_maps_available();
+}
 
 // Shape checks of a backward record; fills p (pointers only when need_ptrs).
 hils_status bwd_problem(const hils_backward_args *a, BwdParams *p, bool need_ptrs,
@@ -662,7 +694,22 @@ hils_status bwd_problem(const hils_backward_args *a, BwdParams *p, bool need_ptr
     p->S = a->S; p->W = a->W; p->K = a->K; p->nC = a->N / a->S;
     p->inv_sqrt_d = (float)(1.0 / sqrt((double)a->d));
     const size_t rows = (size_t)a->B * a->Hq * a->N;
-    const size_t need = (rows * 2 + rows * (size_t)a->K * 3) * sizeof(float);
+    // rowstat, chunkstat, then (tensor-core key side) the inverse index
+    size_t need = round256(rows * 2 * sizeof(float)) +
+                  round256(rows * (size_t)a->K * 4 * sizeof(float));
+    const bool tc = keys_tc_ok(a, G, a->N / a->S);
+    BwdIndexParams ip{};
+    int64_t max_units = 0, nbt = 0;
+    if (tc) {
+        bwd_index_shape(a->N, a->N / a->S, &ip);
+        max_units = bwd_keys_max_units(a->B, a->Hkv, a->N, a->S, a->W, a->K, G);
+        nbt = (int64_t)a->B * a->Hkv * ((a->N + 127) / 128);
+        need += round256((size_t)a->B * a->Hkv * ip.off_stride * sizeof(int)) +
+                round256((size_t)a->B * a->Hkv * a->N * a->K * sizeof(int32_t)) +
+                round256((size_t)max_units * sizeof(int2)) +
+                round256((size_t)nbt * 2 * sizeof(int) + sizeof(int)) +
+                round256((size_t)max_units * bwd_keys_partial_floats(a->d) * sizeof(float));
+    }
     if (ws_bytes) *ws_bytes = need;
     if (!need_ptrs) return HILS_OK;
     if (!a->Q || !a->Kc || !a->V || !a->dO || !a->idx || !a->dQ || !a->dK || !a->dV)
@@ -680,8 +727,27 @@ hils_status bwd_problem(const hils_backward_args *a, BwdParams *p, bool need_ptr
     p->dO = a->dO; p->bias = a->bias; p->idx = a->idx;
     p->dQ = a->dQ; p->dQs = a->dQs; p->dK = a->dK; p->dV = a->dV;
     p->dKlm = a->dKlm; p->dbias = a->dbias;
-    p->rowstat = (float *)a->workspace;
-    p->chunkstat = p->rowstat + rows * 2;
+    uint8_t *w = (uint8_t *)a->workspace;
+    p->rowstat = (float *)w;
+    w += round256(rows * 2 * sizeof(float));
+    p->chunkstat = (float *)w;
+    w += round256(rows * (size_t)a->K * 4 * sizeof(float));
+    p->tc_keys = tc;
+    if (tc) {
+        p->csr_off = (int *)w;
+        w += round256((size_t)a->B * a->Hkv * ip.off_stride * sizeof(int));
+        p->csr_ent = (int32_t *)w;
+        w += round256((size_t)a->B * a->Hkv * a->N * a->K * sizeof(int32_t));
+        p->units = (int2 *)w;
+        w += round256((size_t)max_units * sizeof(int2));
+        p->nunits_blk = (int *)w;
+        p->tickets = p->nunits_blk + nbt;
+        p->n_units = p->tickets + nbt;
+        w += round256((size_t)nbt * 2 * sizeof(int) + sizeof(int));
+        p->partial = (float *)w;
+        p->max_units = max_units;
+    }
+    p->status = a->status;
     return HILS_OK;
 }
 
@@ -707,6 +773,38 @@ extern "C" hils_status hils_bwd_prefill(const hils_backward_args *a, void *strea
     if (s != HILS_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;
+    if (p.tc_keys) {
+        e = a->d == 128 ? launch_rows_d<__nv_bfloat16, 128>(p, st)
+                        : launch_rows_d<__nv_bfloat16, 64>(p, st);
+        count_launches(1);
+        if (e != cudaSuccess) return HILS_ERR_CUDA;
+        BwdIndexParams ip{};
+        bwd_index_shape(p.N, p.nC, &ip);
+        ip.idx = p.idx; ip.off = p.csr_off; ip.ent = p.csr_ent;
+        ip.ent_stride = (int64_t)p.N * p.K;
+        ip.BH = p.B * p.Hkv; ip.N = p.N; ip.S = p.S; ip.W = p.W; ip.K = p.K;
+        if (p.nC > 0) {
+            e = launch_bwd_index(ip, st);
+            if (e != cudaSuccess) return HILS_ERR_CUDA;
+        }
+        BwdTcParams tp{};
+        tp.Q = p.Q; tp.Qs = p.Qs; tp.Kc = p.Kc; tp.V = p.Vc; tp.dO = p.dO;
+        tp.rowstat = p.rowstat; tp.chunkstat = p.chunkstat;
+        tp.off = p.csr_off; tp.ent = p.csr_ent;
+        tp.dK = p.dK; tp.dV = p.dV; tp.dKlm = p.dKlm; tp.dbias = p.dbias;
+        tp.status = p.status;
+        tp.units = p.units; tp.nunits_blk = p.nunits_blk; tp.tickets = p.tickets;
+        tp.n_units = p.n_units; tp.partial = p.partial; tp.max_units = p.max_units;
+        tp.unit_batches = bwd_keys_unit_batches(p.B, p.Hkv, p.N, p.S, p.W, p.K, p.G);
+        tp.off_stride = ip.off_stride; tp.ent_stride = ip.ent_stride;
+        tp.B = p.B; tp.Hq = p.Hq; tp.Hkv = p.Hkv; tp.G = p.G; tp.N = p.N;
+        tp.d = a->d; tp.S = p.S; tp.W = p.W; tp.K = p.K;
+        tp.nC = p.nC > 0 ? p.nC : 0; tp.nseg = ip.nseg;
+        tp.inv_sqrt_d = p.inv_sqrt_d;
+        for (int k = 0; k < kMaxHeads; ++k) tp.group_heads[k] = p.group_heads[k];
+        e = launch_bwd_keys_tc(tp, st);
+        return e == cudaSuccess ? HILS_OK : HILS_ERR_CUDA;
+    }
     if (a->dtype == HILS_BF16)
         e = a->d == 128 ? launch_bwd_d<__nv_bfloat16, 128>(p, st)
                         : launch_bwd_d<__nv_bfloat16, 64>(p, st);

@@ -81,6 +81,13 @@ bool attend_supported(const Problem &p) {
 }  // namespace
 
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n); }
+
+bool tc_make_map(CUtensorMap *m, const void *base, int d, int64_t rows, int d2,
+                 int d3, int box_rows) {
+    return make_map(m, base, d, rows, d2, d3, box_rows);
+}
+
+bool tc_maps_available() { return encode_fn() != nullptr; }
 uint64_t launch_total() { return g_launches.load(); }
 
 bool fast_path_supported(const Problem &p) {

@@ -302,6 +302,7 @@ typedef struct {
     float *dQ, *dQs, *dK, *dV, *dKlm, *dbias;
     void *workspace;
     size_t workspace_bytes;
+    int32_t *status;                /* device, nullable */
 } hils_backward_args;
 
 hils_status hils_bwd_prefill_workspace_size(const hils_backward_args *args,

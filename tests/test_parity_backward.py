@@ -1,9 +1,15 @@
 """GPU parity of hils_bwd_prefill (through the C ABI) against the fp64
 backward oracle, on the selection the GPU forward made.
 
-Tolerance: the GPU gets the same (bf16- or f32-exact) inputs as the oracle
-and differs only by f32 rounding in sums of at most a few thousand terms
-(~n * 2^-24 < 2e-4 relative to the largest entry of each gradient)."""
+Tolerances, relative to the largest entry of each gradient:
+- f32 arithmetic throughout (f32 inputs; dQ, dKlm, dbias for bf16 inputs):
+  the GPU gets the same inputs as the oracle and differs only by f32
+  rounding in sums of at most a few thousand terms, ~n * 2^-24 < 2e-4.
+- dK, dV for bf16 inputs: the tensor-core key side rounds the weights p_j
+  and ds_j to bf16 before the products (relative error <= 2^-9 per term,
+  independent across terms), so a sum's error is about 2^-9 times the
+  root-sum-square of its terms, which for these random inputs is at most
+  the sum's own scale; 2^-8 = 3.9e-3 leaves a factor of two."""
 import numpy as np
 import pytest
 import torch
@@ -15,6 +21,7 @@ from oracle.backward import hils_backward
 pytestmark = pytest.mark.gpu
 
 REL = 2e-4
+REL_BF16_KEYS = 2.0 ** -8
 
 
 def _run(sh, seed, dev):
@@ -41,7 +48,10 @@ def _check(inp, idx, dO, gr, sh):
         got = gr[name].double().cpu().numpy()
         want = ref[name]
         err = np.abs(got - want).max() / max(1e-30, np.abs(want).max())
-        assert err <= REL, f"{name}: rel err {err:.3e}"
+        tol = REL
+        if sh.dtype == "bf16" and name in ("dK", "dV"):
+            tol = REL_BF16_KEYS
+        assert err <= tol, f"{name}: rel err {err:.3e} (tol {tol:.1e})"
 
 
 CASES = {
@@ -51,11 +61,20 @@ CASES = {
     "f32_qcal": synth.Shape("f32", 1, 2, 1, 128, 768, 64, 128, 3, "qcal"),
     "bf16_needles": synth.Shape("bf16", 1, 4, 1, 128, 2048, 64, 256, 8,
                                 "needles", n_needles=3),
-    # 128-token chunks: the key side works in 64-token blocks, two per chunk
+    # 128-token chunks
     "bf16_S128_g4_d128_ragged": synth.Shape("bf16", 1, 8, 2, 128, 2500, 128,
                                             300, 6),
     "f32_S128_qcal_d64": synth.Shape("f32", 1, 4, 1, 64, 1300, 128, 200, 4,
                                      "qcal"),
+    # bf16 query calibration: the key side gathers the scoring rows too
+    "bf16_qcal_d128": synth.Shape("bf16", 1, 4, 1, 128, 1300, 64, 200, 6,
+                                  "qcal"),
+    "bf16_S128_qcal_d64": synth.Shape("bf16", 1, 4, 1, 64, 1400, 128, 256, 4,
+                                      "qcal"),
+    # G = 8: eight pairs per row in a batch of 64
+    "bf16_g8_d128": synth.Shape("bf16", 1, 8, 1, 128, 1000, 64, 128, 5),
+    # many key blocks, rows selecting a chunk spread over several batches
+    "bf16_g4_d128_long": synth.Shape("bf16", 1, 4, 1, 128, 3000, 64, 128, 12),
 }
 
 

@@ -774,9 +774,24 @@ extern "C" hils_status hils_bwd_prefill(const hils_backward_args *a, void *strea
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (p.tc_keys) {
-        e = a->d == 128 ? launch_rows_d<__nv_bfloat16, 128>(p, st)
-                        : launch_rows_d<__nv_bfloat16, 64>(p, st);
-        count_launches(1);
+        BwdRowsParams rp{};
+        rp.Q = p.Q; rp.Qs = p.Qs; rp.Kc = p.Kc; rp.V = p.Vc; rp.dO = p.dO; rp.Klm = p.Klm;
+        rp.bias = p.bias; rp.idx = p.idx; rp.rowstat = p.rowstat; rp.chunkstat = p.chunkstat;
+        rp.dQ = p.dQ; rp.dQs = p.dQs; rp.status = p.status;
+        rp.B = p.B; rp.Hq = p.Hq; rp.Hkv = p.Hkv; rp.G = p.G; rp.N = p.N; rp.d = a->d;
+        rp.S = p.S; rp.W = p.W; rp.K = p.K; rp.nC = p.nC > 0 ? p.nC : 0;
+        rp.M = 128 / p.G;
+        const int64_t uc = (int64_t)rp.M * p.K;
+        rp.ucap = (int)(uc < rp.nC ? uc : (rp.nC > 0 ? rp.nC : 1));
+        rp.inv_sqrt_d = p.inv_sqrt_d;
+        for (int k = 0; k < kMaxHeads; ++k) rp.group_heads[k] = p.group_heads[k];
+        if (128 % p.G == 0 && bwd_rows_tc_smem(rp) <= 227 * 1024) {
+            e = launch_bwd_rows_tc(rp, st);
+        } else {
+            e = a->d == 128 ? launch_rows_d<__nv_bfloat16, 128>(p, st)
+                            : launch_rows_d<__nv_bfloat16, 64>(p, st);
+            count_launches(1);
+        }
         if (e != cudaSuccess) return HILS_ERR_CUDA;
         BwdIndexParams ip{};
         bwd_index_shape(p.N, p.nC, &ip);

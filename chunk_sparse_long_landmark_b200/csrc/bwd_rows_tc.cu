@@ -1,0 +1,663 @@
+// bwd_rows_tc.cu -- query side of the prefill backward on the sm_100a tensor
+// cores (bf16 inputs): dQ, and the per-(row, head) statistics the key side
+// consumes.
+//
+// "Hierarchical Sparse Attention Done Right", Sec. 3 (RQ2: the fused
+// chunk-level softmax) and Sec. 4 (native sparse training). For one row i,
+// head h (kv group g), with s_j = q.k_j/sqrt(d), u_j = dO.v_j,
+// s^_c = qs.k'_c/sqrt(d) + b'_c:
+//   lz_c   = log sum_{j in c} e^{s_j},  Ubar_c = sum_{j in c} e^{s_j - lz_c} u_j
+//   L      = log(sum_c e^{s^_c} + sum_win e^{s_j})
+//   D      = sum_c e^{s^_c - L} Ubar_c + sum_win e^{s_j - L} u_j
+//   ds_j   = e^{s_j - a_c} (u_j - Ubar_c), a_c = lz_c - s^_c + L  (chunk c)
+//   ds_j   = e^{s_j - L} (u_j - D)                                 (window)
+//   dq     = sum_j ds_j k_j / sqrt(d);  dsh_c = e^{s^_c - L} (Ubar_c - D)
+//
+// Three kernels:
+//   bwd_sh     s^_c of every valid selection (warp per (b, g, i), lanes
+//              split the dims), into slot 3 of the (row, head, slot) record.
+//   bwd_rows   one CTA per (b, g, 128/G adjacent queries) x G heads = 128
+//              rows (row = TMEM lane), like the forward's attention: the
+//              union of the queries' selected chunks and the aligned window,
+//              in 64-token tiles (a 128-token chunk is two), each brought in
+//              by TMA. Two passes over the tiles:
+//                A: S = Q K^T, U = dO V^T (tcgen05.mma, f32 in TMEM) give
+//                   lz_c, Ubar_c of the selected chunks and the window sums;
+//                   then L, D, a_c and dsh_c per row.
+//                B: S, U again; dS (bf16) over the S columns; dQ += dS K
+//                   (tcgen05.mma, A from TMEM, f32 accumulator in TMEM).
+//              Writes dQ (the part through the tokens), L and D, and
+//              (a_c, Ubar_c, dsh_c, s^_c) per selected slot.
+//   bwd_dqs    dqs = sum_c dsh_c k'_c / sqrt(d) per (row, head): into dQs
+//              under query calibration, else added to dQ.
+// Warp roles of bwd_rows: warp 0 TMA producer (K, V), warp 1 MMA issuer and
+// TMEM owner, warps 2-5 Q / dO loader and softmax (warp w reads TMEM lanes
+// 32*(w%4)..+31). Every wait is bounded; a lost arrival ends the kernel
+// with HILS_ERR_DEVICE_TIMEOUT in the status word. No floating-point
+// atomics: every sum has one fixed order.
+#include <math.h>
+
+#include "hils_fast.cuh"
+#include "sm100.cuh"
+#include "tc_kernels.cuh"
+
+namespace hils {
+
+namespace {
+
+using namespace sm100;
+
+constexpr int kRT = 192;          // threads of bwd_rows
+constexpr int kRows = 128;
+constexpr int kTile = 64;         // tokens per tile
+constexpr int kRStg = 3;          // K / V stages
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// ------------------------------------------------------------------ s^_c
+template <int D>
+__global__ void __launch_bounds__(128) bwd_sh_kernel(const BwdRowsParams p) {
+    constexpr int DL = D / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 4 + warp;      // (b, g, i)
+    if (row >= (int64_t)p.B * p.Hkv * p.N) return;
+    const int i = (int)(row % p.N);
+    const int g = (int)((row / p.N) % p.Hkv);
+    const int b = (int)(row / ((int64_t)p.N * p.Hkv));
+    const int64_t bg = (int64_t)b * p.Hkv + g;
+    const __nv_bfloat16 *Qs = reinterpret_cast<const __nv_bfloat16 *>(p.Qs ? p.Qs : p.Q);
+    const __nv_bfloat16 *Kl = reinterpret_cast<const __nv_bfloat16 *>(p.Klm);
+    int64_t w0, nc;
+    window_bounds(i, p.S, p.W, &w0, &nc);
+    float q[8][DL];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+        if (h >= p.G) break;
+        const __nv_bfloat16 *qr = Qs + (((int64_t)b * p.Hq + p.group_heads[g * p.G + h]) * p.N + i) * D +
+                                  lane * DL;
+#pragma unroll
+        for (int r = 0; r < DL; ++r) q[h][r] = __bfloat162float(qr[r]);
+    }
+    const int32_t *ir = p.idx + (bg * p.N + i) * p.K;
+    for (int k = 0; k < p.K; ++k) {
+        const int c = __ldg(ir + k);
+        if (c < 0 || c >= nc) continue;              // uniform over the warp
+        const __nv_bfloat16 *kr = Kl + (bg * p.nC + c) * D + lane * DL;
+        float kv[DL];
+#pragma unroll
+        for (int r = 0; r < DL; ++r) kv[r] = __bfloat162float(kr[r]);
+        const float bc = __ldg(p.bias + bg * p.nC + c);
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+            if (h >= p.G) break;
+            float a = 0.f;
+#pragma unroll
+            for (int r = 0; r < DL; ++r) a = fmaf(q[h][r], kv[r], a);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+            if (lane == 0) {
+                const int64_t rq = ((int64_t)b * p.Hq + p.group_heads[g * p.G + h]) * p.N + i;
+                p.chunkstat[(rq * p.K + k) * 4 + 3] = a * p.inv_sqrt_d + bc;
+            }
+        }
+    }
+}
+
+// --------------------------------------------------------------- dqs
+template <int D>
+__global__ void __launch_bounds__(128) bwd_dqs_kernel(const BwdRowsParams p) {
+    constexpr int DL = D / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 4 + warp;      // (b, g, i)
+    if (row >= (int64_t)p.B * p.Hkv * p.N) return;
+    const int i = (int)(row % p.N);
+    const int g = (int)((row / p.N) % p.Hkv);
+    const int b = (int)(row / ((int64_t)p.N * p.Hkv));
+    const int64_t bg = (int64_t)b * p.Hkv + g;
+    const __nv_bfloat16 *Kl = reinterpret_cast<const __nv_bfloat16 *>(p.Klm);
+    int64_t w0, nc;
+    window_bounds(i, p.S, p.W, &w0, &nc);
+    float acc[8][DL];
+#pragma unroll
+    for (int h = 0; h < 8; ++h)
+#pragma unroll
+        for (int r = 0; r < DL; ++r) acc[h][r] = 0.f;
+    const int32_t *ir = p.idx + (bg * p.N + i) * p.K;
+    for (int k = 0; k < p.K; ++k) {
+        const int c = __ldg(ir + k);
+        if (c < 0 || c >= nc) continue;
+        const __nv_bfloat16 *kr = Kl + (bg * p.nC + c) * D + lane * DL;
+        float kv[DL];
+#pragma unroll
+        for (int r = 0; r < DL; ++r) kv[r] = __bfloat162float(kr[r]);
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+            if (h >= p.G) break;
+            const int64_t rq = ((int64_t)b * p.Hq + p.group_heads[g * p.G + h]) * p.N + i;
+            const float dsh = p.chunkstat[(rq * p.K + k) * 4 + 2];
+#pragma unroll
+            for (int r = 0; r < DL; ++r) acc[h][r] = fmaf(dsh, kv[r], acc[h][r]);
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+        if (h >= p.G) break;
+        const int64_t rq = ((int64_t)b * p.Hq + p.group_heads[g * p.G + h]) * p.N + i;
+        if (p.dQs) {
+            float *o = p.dQs + rq * D + lane * DL;
+#pragma unroll
+            for (int r = 0; r < DL; ++r) o[r] = acc[h][r] * p.inv_sqrt_d;
+        } else {
+            float *o = p.dQ + rq * D + lane * DL;
+#pragma unroll
+            for (int r = 0; r < DL; ++r) o[r] += acc[h][r] * p.inv_sqrt_d;
+        }
+    }
+}
+
+// ---------------------------------------------------------------- rows
+template <int D>
+struct RowLayout {
+    static constexpr uint32_t Q_BYTES = kRows * D * 2;        // Q or dO rows
+    static constexpr uint32_t KV_BYTES = kTile * D * 2;       // K or V tile
+    static constexpr uint32_t OFF_Q = 0;
+    static constexpr uint32_t OFF_O = Q_BYTES;                // dO
+    static constexpr uint32_t OFF_K = 2 * Q_BYTES;
+    static constexpr uint32_t OFF_V = OFF_K + kRStg * KV_BYTES;
+    static constexpr uint32_t OFF_SMALL = OFF_V + kRStg * KV_BYTES;
+    // TMEM: dQ [0, D); buffer sb: S at BUF + 128 sb, U at BUF + 128 sb + 64
+    static constexpr int TM_DQ = 0, TM_BUF = D;
+    static constexpr uint32_t TMEM_COLS = 512u;
+};
+
+struct RowSmall {
+    uint64_t q_full;
+    uint64_t full[kRStg];
+    uint64_t empty[kRStg];
+    uint64_t s_full[2];
+    uint64_t p_full[2];
+    uint64_t buf_free[2];
+    uint64_t acc_done;
+    uint32_t tmem_base;
+    int abort;
+    int n_union;
+    int n_win;
+    int win_start;
+};
+
+__device__ __forceinline__ float row_max64(const uint32_t *r) {
+    float m[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m[k] = __uint_as_float(r[k]);
+#pragma unroll
+    for (int j = 4; j < 64; j += 4)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) m[k] = fmaxf(m[k], __uint_as_float(r[j + k]));
+    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+template <int D>
+__global__ void __launch_bounds__(kRT, 1)
+bwd_rows_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV,
+                   const BwdRowsParams p) {
+    using L = RowLayout<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    RowSmall &st = *reinterpret_cast<RowSmall *>(smem + L::OFF_SMALL);
+    int *s_idx = reinterpret_cast<int *>(smem + L::OFF_SMALL + sizeof(RowSmall));
+    int *s_union = s_idx + p.M * p.K;
+    uint32_t *s_bits = reinterpret_cast<uint32_t *>(s_union + p.ucap);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nqb = (p.N + p.M - 1) / p.M;
+    const int qb = blockIdx.x % nqb;
+    const int g = (blockIdx.x / nqb) % p.Hkv;
+    const int b = blockIdx.x / (nqb * p.Hkv);
+    const int i0 = qb * p.M;
+    const int i_last = min(i0 + p.M, p.N) - 1;
+    const int HT = p.S / kTile;                      // tiles per chunk
+    volatile int *abort = &st.abort;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&st.q_full, 128);
+        for (int s = 0; s < kRStg; ++s) {
+            mbar_init(&st.full[s], 1);
+            mbar_init(&st.empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&st.s_full[s], 1);
+            mbar_init(&st.p_full[s], 128);
+            mbar_init(&st.buf_free[s], 1);
+        }
+        mbar_init(&st.acc_done, 1);
+        st.abort = (p.status && *(volatile int32_t *)p.status ==
+                                    HILS_ERR_DEVICE_TIMEOUT) ? 1 : 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) tmem_alloc(&st.tmem_base, L::TMEM_COLS);
+    // selected chunks of the block's queries -> smem [K][M]; union bitmap
+    const int nwords = (p.nC + 31) >> 5;
+    for (int w = threadIdx.x; w < nwords; w += kRT) s_bits[w] = 0u;
+    __syncthreads();
+    {
+        const int32_t *gidx = p.idx + (((int64_t)b * p.Hkv + g) * p.N + i0) * p.K;
+        const int nvalid = (i_last - i0 + 1) * p.K;
+        for (int e = threadIdx.x; e < p.M * p.K; e += kRT) {
+            const int m = e / p.K, k = e % p.K;
+            int c = e < nvalid ? __ldg(gidx + e) : -1;
+            if (c >= 0) {
+                int64_t w0, nc;
+                window_bounds(i0 + m, p.S, p.W, &w0, &nc);
+                if (c >= nc) c = -1;
+            }
+            s_idx[k * p.M + m] = c;
+            if (c >= 0) atomicOr(&s_bits[c >> 5], 1u << (c & 31));
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {                       // ascending compaction of the union
+        int base = 0;
+        for (int w0i = 0; w0i < nwords; w0i += 32) {
+            const int w = w0i + lane;
+            uint32_t bits = w < nwords ? s_bits[w] : 0u;
+            const int cnt = __popc(bits);
+            int incl = cnt;
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int pos = base + incl - cnt;
+            while (bits) {
+                const int bit = __ffs(bits) - 1;
+                bits &= bits - 1;
+                if (pos < p.ucap) s_union[pos] = w * 32 + bit;
+                ++pos;
+            }
+            base += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            st.n_union = min(base, p.ucap);
+            int64_t w0, nc;
+            window_bounds(i0, p.S, p.W, &w0, &nc);
+            st.win_start = (int)w0;
+            st.n_win = (i_last - (int)w0) / kTile + 1;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = st.tmem_base;
+    const int U = st.n_union;
+    const int NT = U * HT + st.n_win;                // tiles of one pass
+    const int NS = st.abort ? 0 : 2 * NT;            // steps: pass A, pass B
+    const int wstart = st.win_start;
+    auto tile_row = [&](int t) -> int {              // first token of tile t
+        return t < U * HT ? s_union[t / HT] * p.S + (t % HT) * kTile
+                          : wstart + (t - U * HT) * kTile;
+    };
+
+    if (NS == 0) {
+        // skipped: straight to teardown
+    } else if (warp == 0) {
+        // ------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tmK);
+            prefetch_tmap(&tmV);
+            int n = 0;
+            for (; n < NS; ++n) {
+                const int s = n % kRStg;
+                if (n >= kRStg && !mbar_wait(&st.empty[s], ((n / kRStg) - 1) & 1, abort)) break;
+                const int row = tile_row(n % NT);
+                mbar_expect_tx(&st.full[s], 2 * L::KV_BYTES);
+                for (int dh = 0; dh < D / 64; ++dh) {
+                    tma_load_4d(smem + L::OFF_K + s * L::KV_BYTES + dh * (kTile * 128), &tmK,
+                                &st.full[s], dh * 64, row, g, b);
+                    tma_load_4d(smem + L::OFF_V + s * L::KV_BYTES + dh * (kTile * 128), &tmV,
+                                &st.full[s], dh * 64, row, g, b);
+                }
+            }
+            if (*abort)
+                for (int t = (n > kRStg ? n - kRStg : 0); t < n; ++t)
+                    mbar_drain(&st.full[t % kRStg], (t / kRStg) & 1);
+        }
+    } else if (warp == 1) {
+        // ----------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_s = idesc_bf16(kRows, kTile, false);
+            constexpr uint32_t id_q = idesc_bf16(kRows, D, true);
+            const uint32_t sQ = smem_u32(smem + L::OFF_Q);
+            const uint32_t sO = smem_u32(smem + L::OFF_O);
+            const uint32_t sK = smem_u32(smem + L::OFF_K);
+            const uint32_t sV = smem_u32(smem + L::OFF_V);
+            bool ok = mbar_wait(&st.q_full, 0, abort);
+            int ndq = 0;                             // dQ products issued
+            // step u's buffer is released once the softmax warps are done
+            // with it; in pass B after dQ += dS K has consumed dS
+            auto finish = [&](int u) -> bool {
+                const int sb = u & 1, s = u % kRStg;
+                if (!mbar_wait(&st.p_full[sb], (u >> 1) & 1, abort)) return false;
+                tc_fence_after();
+                if (u >= NT) {
+#pragma unroll
+                    for (int kk = 0; kk < kTile / 16; ++kk) {
+                        const uint64_t bk = desc_sw128(sK + s * L::KV_BYTES + kk * 16 * 128,
+                                                       kTile * 128, 1024);
+                        mma_ts(tmem + L::TM_DQ, tmem + L::TM_BUF + sb * 128 + kk * 8, bk, id_q,
+                               (ndq > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    ++ndq;
+                }
+                mma_commit(&st.buf_free[sb]);
+                mma_commit(&st.empty[s]);
+                return true;
+            };
+            for (int n = 0; ok && n < NS; ++n) {
+                const int s = n % kRStg, sb = n & 1;
+                if (!mbar_wait(&st.full[s], (n / kRStg) & 1, abort)) { ok = false; break; }
+                if (n >= 2 && !mbar_wait(&st.buf_free[sb], ((n >> 1) - 1) & 1, abort)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t aq = desc_sw128(sQ + (kk / 4) * (kRows * 128) + (kk % 4) * 32, 16, 1024);
+                    const uint64_t bk = desc_sw128(sK + s * L::KV_BYTES + (kk / 4) * (kTile * 128) +
+                                                       (kk % 4) * 32, 16, 1024);
+                    mma_ss(tmem + L::TM_BUF + sb * 128, aq, bk, id_s, kk > 0 ? 1u : 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t ao = desc_sw128(sO + (kk / 4) * (kRows * 128) + (kk % 4) * 32, 16, 1024);
+                    const uint64_t bv = desc_sw128(sV + s * L::KV_BYTES + (kk / 4) * (kTile * 128) +
+                                                       (kk % 4) * 32, 16, 1024);
+                    mma_ss(tmem + L::TM_BUF + sb * 128 + 64, ao, bv, id_s, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&st.s_full[sb]);
+                if (n >= 1 && !finish(n - 1)) { ok = false; break; }
+            }
+            if (ok) finish(NS - 1);
+            mma_commit(&st.acc_done);
+            mbar_drain(&st.acc_done, 0);
+        }
+    } else {
+        // -------------------------------------------- softmax / epilogue
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const int m = r / p.G, hh = r % p.G;
+        const int i = i0 + m;
+        const bool valid = i < p.N;
+        const int h = p.group_heads[g * p.G + hh];
+        const int64_t rq = ((int64_t)b * p.Hq + h) * p.N + (valid ? i : 0);
+        float *cs = p.chunkstat + rq * p.K * 4;      // this row's slot records
+        int64_t w0 = 0, nc = 0;
+        if (valid) window_bounds(i, p.S, p.W, &w0, &nc);
+
+        // Q and dO rows -> shared memory (A operands: K-major, 128-byte
+        // swizzle), 16-byte units
+        {
+            constexpr int UPR = D / 8;
+            const int tid = threadIdx.x - 64;
+            const __nv_bfloat16 *Qp = reinterpret_cast<const __nv_bfloat16 *>(p.Q);
+            const __nv_bfloat16 *Op = reinterpret_cast<const __nv_bfloat16 *>(p.dO);
+#pragma unroll 1
+            for (int arr = 0; arr < 2; ++arr) {
+                const __nv_bfloat16 *src = arr == 0 ? Qp : Op;
+                uint8_t *dstb = smem + (arr == 0 ? L::OFF_Q : L::OFF_O);
+#pragma unroll 1
+                for (int e0 = 0; e0 < kRows * UPR; e0 += 8 * 128) {
+                    uint4 v[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const int e = e0 + q * 128 + tid;
+                        const int rr = e / UPR, u = e % UPR;
+                        const int mi = i0 + rr / p.G;
+                        v[q] = make_uint4(0u, 0u, 0u, 0u);
+                        if (e < kRows * UPR && mi < p.N) {
+                            const int hq = p.group_heads[g * p.G + rr % p.G];
+                            v[q] = __ldg(reinterpret_cast<const uint4 *>(
+                                       src + (((int64_t)b * p.Hq + hq) * p.N + mi) * D) + u);
+                        }
+                    }
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const int e = e0 + q * 128 + tid;
+                        if (e >= kRows * UPR) continue;
+                        const int rr = e / UPR, u = e % UPR;
+                        *reinterpret_cast<uint4 *>(dstb + (u >> 3) * (kRows * 128) + rr * 128 +
+                                                   (((u & 7) ^ (rr & 7)) << 4)) = v[q];
+                    }
+                }
+            }
+            fence_async_smem();
+            mbar_arrive(&st.q_full);
+        }
+
+        const int *myidx = s_idx + m;                // stride M
+        const int M_ = p.M;
+        const float sl2 = p.inv_sqrt_d * kLog2e;
+        const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+        // pass A state: the current chunk's (max, sum, sum * u) in log2
+        // units; the window's
+        float cm = -INFINITY, cz = 0.f, czu = 0.f;
+        float wm = -INFINITY, wz = 0.f, wzu = 0.f;
+        float Lr = 0.f, Dr = 0.f, L2 = 0.f;
+        int kp = 0;                                  // position in this row's selection
+        float a2 = 0.f, ub = 0.f;                    // pass B: current chunk's a (log2), Ubar
+        bool ok = true;
+
+        for (int n = 0; n < NS; ++n) {
+            const int sb = n & 1;
+            const bool passB = n >= NT;
+            const int t = passB ? n - NT : n;
+            if (n == NT) {
+                // ---- between the passes: L, D; a_c and dsh_c per slot
+                if (valid) {
+                    float top = wm;                  // the window holds token i
+                    for (int k = 0; k < p.K; ++k)
+                        if (myidx[k * M_] >= 0) top = fmaxf(top, cs[k * 4 + 3] * kLog2e);
+                    float tot = wz * fast_exp2(wm - top);
+                    for (int k = 0; k < p.K; ++k)
+                        if (myidx[k * M_] >= 0) tot += fast_exp2(cs[k * 4 + 3] * kLog2e - top);
+                    L2 = top + __log2f(tot);
+                    float Dv = wzu * fast_exp2(wm - L2);
+                    for (int k = 0; k < p.K; ++k)
+                        if (myidx[k * M_] >= 0) Dv += fast_exp2(cs[k * 4 + 3] * kLog2e - L2) * cs[k * 4 + 1];
+                    Lr = L2 * kLn2;
+                    Dr = Dv;
+                    for (int k = 0; k < p.K; ++k) {
+                        if (myidx[k * M_] < 0) continue;
+                        const float lz = cs[k * 4], ubk = cs[k * 4 + 1], sh = cs[k * 4 + 3];
+                        cs[k * 4] = lz - sh + Lr;
+                        cs[k * 4 + 2] = fast_exp2((sh - Lr) * kLog2e) * (ubk - Dr);
+                    }
+                    p.rowstat[rq * 2] = Lr;
+                    p.rowstat[rq * 2 + 1] = Dr;
+                }
+                kp = 0;
+            }
+            if (!__all_sync(0xffffffffu, mbar_wait(&st.s_full[sb], (n >> 1) & 1, abort))) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t tS = trow + L::TM_BUF + sb * 128;
+            // does this row's query select the tile's chunk (chunk tiles)
+            bool sel = false;
+            bool first = false, last = false;
+            int kslot = 0;
+            if (t < U * HT) {
+                const int c = s_union[t / HT];
+                first = (t % HT) == 0;
+                last = (t % HT) == HT - 1;
+                int ck = kp < p.K ? myidx[kp * M_] : 0x7fffffff;
+                while (kp < p.K && (ck < c)) {
+                    ++kp;
+                    ck = kp < p.K ? myidx[kp * M_] : 0x7fffffff;
+                }
+                sel = valid && kp < p.K && ck == c;
+                kslot = kp;
+                if (sel && last) ++kp;
+            }
+            const int j0 = t - U * HT >= 0 ? wstart + (t - U * HT) * kTile : 0;
+            const bool win = t >= U * HT;
+            const bool edge = win && (!valid || j0 < w0 || j0 + kTile - 1 > i);
+            const bool any_edge = __any_sync(0xffffffffu, edge);
+            const bool need = win ? true : __any_sync(0xffffffffu, sel);
+            if (!passB) {
+                // ------------------------------------------------ pass A
+                if (need) {
+                    uint32_t sr[64], ur[64];
+                    tmem_ld32(tS, sr);
+                    tmem_ld32(tS + 32, sr + 32);
+                    tmem_ld32(tS + 64, ur);
+                    tmem_ld32(tS + 96, ur + 32);
+                    tmem_wait_ld();
+                    if (win && any_edge) {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) {
+                            const int pos = j0 + j;
+                            const bool in = valid && pos >= w0 && pos <= i;
+                            sr[j] = in ? sr[j] : __float_as_uint(-INFINITY);
+                        }
+                    }
+                    if (win || sel) {
+                        const float mx = row_max64(sr) * sl2;
+                        float &M = win ? wm : cm;
+                        float &Z = win ? wz : cz;
+                        float &ZU = win ? wzu : czu;
+                        if (!win && first) { M = -INFINITY; Z = 0.f; ZU = 0.f; }
+                        const float mn = fmaxf(M, mx);
+                        if (mn != -INFINITY) {
+                            const float f = fast_exp2(M - mn);
+                            float z4[4] = {0.f, 0.f, 0.f, 0.f}, zu4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                            for (int j = 0; j < 64; ++j) {
+                                const float e = fast_exp2(fmaf(__uint_as_float(sr[j]), sl2, -mn));
+                                z4[j & 3] += e;
+                                zu4[j & 3] = fmaf(e, __uint_as_float(ur[j]), zu4[j & 3]);
+                            }
+                            Z = Z * f + ((z4[0] + z4[1]) + (z4[2] + z4[3]));
+                            ZU = ZU * f + ((zu4[0] + zu4[1]) + (zu4[2] + zu4[3]));
+                            M = mn;
+                        }
+                        if (!win && last) {          // lz_c (natural log), Ubar_c
+                            cs[kslot * 4] = (cm + __log2f(cz)) * kLn2;
+                            cs[kslot * 4 + 1] = czu / cz;
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&st.p_full[sb]);
+            } else {
+                // ------------------------------------------------ pass B
+                uint32_t pk[32];
+                if (need) {
+                    if (sel && first) {
+                        a2 = cs[kslot * 4] * kLog2e;
+                        ub = cs[kslot * 4 + 1];
+                    }
+                    uint32_t sr[64], ur[64];
+                    tmem_ld32(tS, sr);
+                    tmem_ld32(tS + 32, sr + 32);
+                    tmem_ld32(tS + 64, ur);
+                    tmem_ld32(tS + 96, ur + 32);
+                    tmem_wait_ld();
+                    const float sub = win ? L2 : a2;
+                    const float del = win ? Dr : ub;
+                    const bool act = win ? valid : sel;
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        float2 e = f2_fma(make_float2(__uint_as_float(sr[2 * j]),
+                                                      __uint_as_float(sr[2 * j + 1])),
+                                          make_float2(sl2, sl2), make_float2(-sub, -sub));
+                        e.x = fast_exp2(e.x);
+                        e.y = fast_exp2(e.y);
+                        if (win && any_edge) {
+                            const int pos = j0 + 2 * j;
+                            e.x = (valid && pos >= w0 && pos <= i) ? e.x : 0.f;
+                            e.y = (valid && pos + 1 >= w0 && pos + 1 <= i) ? e.y : 0.f;
+                        }
+                        const float2 du = f2_add(make_float2(__uint_as_float(ur[2 * j]),
+                                                             __uint_as_float(ur[2 * j + 1])),
+                                                 make_float2(-del, -del));
+                        const float2 ds = f2_mul(e, du);
+                        pk[j] = act ? pack_bf16(ds.x, ds.y) : 0u;
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) pk[j] = 0u;
+                }
+                tmem_st32(tS, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&st.p_full[sb]);
+            }
+        }
+        // dQ (through the tokens) once the last product is done
+        if (ok && NS > 0) ok = __all_sync(0xffffffffu, mbar_wait(&st.acc_done, 0, abort));
+        if (ok) {
+            tc_fence_after();
+            float *dq = p.dQ + rq * D;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t rv[32];
+                tmem_ld32(trow + L::TM_DQ + c0, rv);     // collective: every lane
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int q = 0; q < 32; q += 4)
+                        *reinterpret_cast<float4 *>(dq + c0 + q) = make_float4(
+                            __uint_as_float(rv[q]) * p.inv_sqrt_d, __uint_as_float(rv[q + 1]) * p.inv_sqrt_d,
+                            __uint_as_float(rv[q + 2]) * p.inv_sqrt_d, __uint_as_float(rv[q + 3]) * p.inv_sqrt_d);
+                }
+            }
+        }
+    }
+
+    // ------------------------------------------------------------ teardown
+    if (*abort && (threadIdx.x & 31) == 0) report(p.status, HILS_ERR_DEVICE_TIMEOUT);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::TMEM_COLS);
+    }
+}
+
+// Shared memory of one CTA, at least 116 KB: two CTAs on one SM would
+// contend for its 512 TMEM columns.
+template <int D>
+size_t rows_smem(const BwdRowsParams &p) {
+    size_t small = sizeof(RowSmall) + sizeof(int) * ((size_t)p.M * p.K + p.ucap) +
+                   sizeof(uint32_t) * (((size_t)p.nC + 31) / 32);
+    const size_t n = 1024 + RowLayout<D>::OFF_SMALL + ((small + 15) / 16) * 16;
+    return n < 116 * 1024 ? 116 * 1024 : n;
+}
+
+template <int D>
+cudaError_t launch_rows_tc_t(const BwdRowsParams &p, cudaStream_t st) {
+    CUtensorMap mk, mv;
+    if (!tc_make_map(&mk, p.Kc, D, p.N, p.Hkv, p.B, kTile) ||
+        !tc_make_map(&mv, p.V, D, p.N, p.Hkv, p.B, kTile))
+        return cudaErrorInvalidValue;
+    const int64_t rows = (int64_t)p.B * p.Hkv * p.N;
+    const unsigned wgrid = (unsigned)((rows + 3) / 4);
+    if (p.nC > 0) bwd_sh_kernel<D><<<wgrid, 128, 0, st>>>(p);
+    const size_t smem = rows_smem<D>(p);
+    auto kern = bwd_rows_tc_kernel<D>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int nqb = (p.N + p.M - 1) / p.M;
+    kern<<<(unsigned)((int64_t)p.B * p.Hkv * nqb), kRT, smem, st>>>(mk, mv, p);
+    if (p.nC > 0 || p.dQs) bwd_dqs_kernel<D><<<wgrid, 128, 0, st>>>(p);
+    count_launches(1 + (p.nC > 0 ? 1 : 0) + ((p.nC > 0 || p.dQs) ? 1 : 0));
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t bwd_rows_tc_smem(const BwdRowsParams &p) {
+    return p.d == 128 ? rows_smem<128>(p) : rows_smem<64>(p);
+}
+
+cudaError_t launch_bwd_rows_tc(const BwdRowsParams &p, cudaStream_t st) {
+    return p.d == 128 ? launch_rows_tc_t<128>(p, st) : launch_rows_tc_t<64>(p, st);
+}
+
+}  // namespace hils

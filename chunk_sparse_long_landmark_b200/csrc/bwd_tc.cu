@@ -733,11 +733,20 @@ bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap tmK,
     }
 }
 
+// Shared memory of one CTA, at least 116 KB: two CTAs on one SM would
+// contend for its 512 TMEM columns.
+template <int D, bool QCAL>
+constexpr size_t keys_smem() {
+    return 1024 + KeyLayout<D, QCAL>::OFF_SMALL + sizeof(KeySmall<D, KeyLayout<D, QCAL>::NSTG>) <
+                   116 * 1024
+               ? 116 * 1024
+               : 1024 + KeyLayout<D, QCAL>::OFF_SMALL + sizeof(KeySmall<D, KeyLayout<D, QCAL>::NSTG>);
+}
+
 template <int D, bool QCAL>
 cudaError_t launch_keys_tc_t(const BwdTcParams &p, const CUtensorMap &mk,
                              const CUtensorMap &mv, cudaStream_t stream) {
-    using L = KeyLayout<D, QCAL>;
-    const size_t smem = 1024 + L::OFF_SMALL + sizeof(KeySmall<D, L::NSTG>);
+    const size_t smem = keys_smem<D, QCAL>();
     auto kern = bwd_keys_tc_kernel<D, QCAL>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -746,10 +755,6 @@ cudaError_t launch_keys_tc_t(const BwdTcParams &p, const CUtensorMap &mk,
     return cudaGetLastError();
 }
 
-template <int D, bool QCAL>
-constexpr size_t keys_smem() {
-    return 1024 + KeyLayout<D, QCAL>::OFF_SMALL + sizeof(KeySmall<D, KeyLayout<D, QCAL>::NSTG>);
-}
 
 }  // namespace
 

@@ -63,6 +63,24 @@ struct BwdTcParams {
     int16_t group_heads[kMaxHeads];
 };
 
+// Query side of the backward on the tensor cores (bf16, 128 % G == 0).
+struct BwdRowsParams {
+    const void *Q, *Qs, *Kc, *V, *dO, *Klm;
+    const float *bias;
+    const int32_t *idx;
+    float *rowstat;           // [B,Hq,N,2]: L, D
+    float *chunkstat;         // [B,Hq,N,K,4]: a, Ubar, dsh, s^
+    float *dQ, *dQs;
+    int32_t *status;
+    int B, Hq, Hkv, G, N, d, S, W, K, nC;
+    int M;                    // queries per CTA: 128 / G
+    int ucap;                 // capacity of the chunk-union list: min(M*K, nC)
+    float inv_sqrt_d;
+    int16_t group_heads[kMaxHeads];
+};
+
+size_t bwd_rows_tc_smem(const BwdRowsParams &p);
+cudaError_t launch_bwd_rows_tc(const BwdRowsParams &p, cudaStream_t st);
 void bwd_index_shape(int N, int nC, BwdIndexParams *ip);
 size_t bwd_keys_tc_smem(int d, bool qcal);
 int64_t bwd_keys_max_units(int B, int Hkv, int N, int S, int W, int K, int G);

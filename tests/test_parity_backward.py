@@ -2,14 +2,14 @@
 backward oracle, on the selection the GPU forward made.
 
 Tolerances, relative to the largest entry of each gradient:
-- f32 arithmetic throughout (f32 inputs; dQ, dKlm, dbias for bf16 inputs):
+- f32 arithmetic throughout (f32 inputs; dQs, dKlm, dbias for bf16 inputs):
   the GPU gets the same inputs as the oracle and differs only by f32
   rounding in sums of at most a few thousand terms, ~n * 2^-24 < 2e-4.
-- dK, dV for bf16 inputs: the tensor-core key side rounds the weights p_j
-  and ds_j to bf16 before the products (relative error <= 2^-9 per term,
-  independent across terms), so a sum's error is about 2^-9 times the
-  root-sum-square of its terms, which for these random inputs is at most
-  the sum's own scale; 2^-8 = 3.9e-3 leaves a factor of two."""
+- dQ, dK, dV for bf16 inputs: the tensor-core kernels round the weights
+  p_j and ds_j to bf16 before the products (relative error <= 2^-9 per
+  term, independent across terms), so a sum's error is about 2^-9 times
+  the root-sum-square of its terms, which for these random inputs is at
+  most the sum's own scale; 2^-8 = 3.9e-3 leaves a factor of two."""
 import numpy as np
 import pytest
 import torch
@@ -21,7 +21,7 @@ from oracle.backward import hils_backward
 pytestmark = pytest.mark.gpu
 
 REL = 2e-4
-REL_BF16_KEYS = 2.0 ** -8
+REL_BF16_TC = 2.0 ** -8
 
 
 def _run(sh, seed, dev):
@@ -49,8 +49,8 @@ def _check(inp, idx, dO, gr, sh):
         want = ref[name]
         err = np.abs(got - want).max() / max(1e-30, np.abs(want).max())
         tol = REL
-        if sh.dtype == "bf16" and name in ("dK", "dV"):
-            tol = REL_BF16_KEYS
+        if sh.dtype == "bf16" and name in ("dQ", "dK", "dV"):
+            tol = REL_BF16_TC
         assert err <= tol, f"{name}: rel err {err:.3e} (tol {tol:.1e})"
 
 

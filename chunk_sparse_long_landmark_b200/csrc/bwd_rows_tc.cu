@@ -32,9 +32,10 @@
 //              under query calibration, else added to dQ.
 // Warp roles of bwd_rows: warp 0 TMA producer (K, V), warp 1 MMA issuer and
 // TMEM owner, warps 2-5 Q / dO loader and softmax (warp w reads TMEM lanes
-// 32*(w%4)..+31). Every wait is bounded; a lost arrival ends the kernel
-// with HILS_ERR_DEVICE_TIMEOUT in the status word. No floating-point
-// atomics: every sum has one fixed order.
+// 32*(w%4)..+31); two CTAs per SM. L and D are summed online during pass A
+// (each selected chunk's record is fetched one chunk ahead). Every wait is
+// bounded; a lost arrival ends the kernel with HILS_ERR_DEVICE_TIMEOUT in the
+// status word. No floating-point atomics: every sum has one fixed order.
 #include <math.h>
 
 #include "hils_fast.cuh"
@@ -50,11 +51,26 @@ using namespace sm100;
 constexpr int kRT = 192;          // threads of bwd_rows
 constexpr int kRows = 128;
 constexpr int kTile = 64;         // tokens per tile
-constexpr int kRStg = 3;          // K / V stages
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+// DL consecutive bf16 values (DL = 2 or 4) in one load, as f32
+template <int DL>
+__device__ __forceinline__ void load_bf16s(const __nv_bfloat16 *src, float *f) {
+    if constexpr (DL == 4) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2 *>(src));
+        f[0] = __uint_as_float(w.x << 16); f[1] = __uint_as_float(w.x & 0xffff0000u);
+        f[2] = __uint_as_float(w.y << 16); f[3] = __uint_as_float(w.y & 0xffff0000u);
+    } else {
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(src));
+        f[0] = __uint_as_float(w << 16); f[1] = __uint_as_float(w & 0xffff0000u);
+    }
+}
+
 // ------------------------------------------------------------------ s^_c
+// Warp per (b, g, i): the row's top-K slots are read 32 at a time (lane =
+// slot) and broadcast; four landmark rows are in flight at once; lanes
+// split the dims of the dot products.
 template <int D>
 __global__ void __launch_bounds__(128) bwd_sh_kernel(const BwdRowsParams p) {
     constexpr int DL = D / 32;
@@ -73,37 +89,49 @@ __global__ void __launch_bounds__(128) bwd_sh_kernel(const BwdRowsParams p) {
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
         if (h >= p.G) break;
-        const __nv_bfloat16 *qr = Qs + (((int64_t)b * p.Hq + p.group_heads[g * p.G + h]) * p.N + i) * D +
-                                  lane * DL;
-#pragma unroll
-        for (int r = 0; r < DL; ++r) q[h][r] = __bfloat162float(qr[r]);
+        load_bf16s<DL>(Qs + (((int64_t)b * p.Hq + p.group_heads[g * p.G + h]) * p.N + i) * D + lane * DL,
+                       q[h]);
     }
     const int32_t *ir = p.idx + (bg * p.N + i) * p.K;
-    for (int k = 0; k < p.K; ++k) {
-        const int c = __ldg(ir + k);
-        if (c < 0 || c >= nc) continue;              // uniform over the warp
-        const __nv_bfloat16 *kr = Kl + (bg * p.nC + c) * D + lane * DL;
-        float kv[DL];
+    for (int k0 = 0; k0 < p.K; k0 += 32) {
+        int cl = k0 + lane < p.K ? __ldg(ir + k0 + lane) : -1;
+        if (cl >= nc) cl = -1;
+        const int kn = min(32, p.K - k0);
+        for (int k1 = 0; k1 < kn; k1 += 4) {
+            float kv[4][DL], bc[4];
+            int cc[4];
 #pragma unroll
-        for (int r = 0; r < DL; ++r) kv[r] = __bfloat162float(kr[r]);
-        const float bc = __ldg(p.bias + bg * p.nC + c);
+            for (int u = 0; u < 4; ++u) {
+                cc[u] = __shfl_sync(0xffffffffu, cl, (k1 + u) & 31);
+                if (k1 + u >= kn) cc[u] = -1;
+                const int c = cc[u] < 0 ? 0 : cc[u];
+                load_bf16s<DL>(Kl + (bg * p.nC + c) * D + lane * DL, kv[u]);
+                bc[u] = __ldg(p.bias + bg * p.nC + c);
+            }
 #pragma unroll
-        for (int h = 0; h < 8; ++h) {
-            if (h >= p.G) break;
-            float a = 0.f;
+            for (int u = 0; u < 4; ++u) {
+                if (cc[u] < 0) continue;             // uniform over the warp
 #pragma unroll
-            for (int r = 0; r < DL; ++r) a = fmaf(q[h][r], kv[r], a);
+                for (int h = 0; h < 8; ++h) {
+                    if (h >= p.G) break;
+                    float a = 0.f;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-            if (lane == 0) {
-                const int64_t rq = ((int64_t)b * p.Hq + p.group_heads[g * p.G + h]) * p.N + i;
-                p.chunkstat[(rq * p.K + k) * 4 + 3] = a * p.inv_sqrt_d + bc;
+                    for (int r = 0; r < DL; ++r) a = fmaf(q[h][r], kv[u][r], a);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+                    if (lane == 0) {
+                        const int64_t rq = ((int64_t)b * p.Hq + p.group_heads[g * p.G + h]) * p.N + i;
+                        p.chunkstat[(rq * p.K + k0 + k1 + u) * 4 + 3] = a * p.inv_sqrt_d + bc[u];
+                    }
+                }
             }
         }
     }
 }
 
 // --------------------------------------------------------------- dqs
+// Same layout: slots 32 at a time, each head's dsh of the slot read by the
+// slot's lane and broadcast, four landmark rows in flight.
 template <int D>
 __global__ void __launch_bounds__(128) bwd_dqs_kernel(const BwdRowsParams p) {
     constexpr int DL = D / 32;
@@ -123,20 +151,38 @@ __global__ void __launch_bounds__(128) bwd_dqs_kernel(const BwdRowsParams p) {
 #pragma unroll
         for (int r = 0; r < DL; ++r) acc[h][r] = 0.f;
     const int32_t *ir = p.idx + (bg * p.N + i) * p.K;
-    for (int k = 0; k < p.K; ++k) {
-        const int c = __ldg(ir + k);
-        if (c < 0 || c >= nc) continue;
-        const __nv_bfloat16 *kr = Kl + (bg * p.nC + c) * D + lane * DL;
-        float kv[DL];
-#pragma unroll
-        for (int r = 0; r < DL; ++r) kv[r] = __bfloat162float(kr[r]);
+    for (int k0 = 0; k0 < p.K; k0 += 32) {
+        int cl = k0 + lane < p.K ? __ldg(ir + k0 + lane) : -1;
+        if (cl >= nc) cl = -1;
+        float dl[8];
 #pragma unroll
         for (int h = 0; h < 8; ++h) {
-            if (h >= p.G) break;
+            dl[h] = 0.f;
+            if (h >= p.G || cl < 0) continue;
             const int64_t rq = ((int64_t)b * p.Hq + p.group_heads[g * p.G + h]) * p.N + i;
-            const float dsh = p.chunkstat[(rq * p.K + k) * 4 + 2];
+            dl[h] = p.chunkstat[(rq * p.K + k0 + lane) * 4 + 2];
+        }
+        const int kn = min(32, p.K - k0);
+        for (int k1 = 0; k1 < kn; k1 += 4) {
+            float kv[4][DL];
+            int cc[4];
 #pragma unroll
-            for (int r = 0; r < DL; ++r) acc[h][r] = fmaf(dsh, kv[r], acc[h][r]);
+            for (int u = 0; u < 4; ++u) {
+                cc[u] = __shfl_sync(0xffffffffu, cl, (k1 + u) & 31);
+                if (k1 + u >= kn) cc[u] = -1;
+                load_bf16s<DL>(Kl + (bg * p.nC + (cc[u] < 0 ? 0 : cc[u])) * D + lane * DL, kv[u]);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+#pragma unroll
+                for (int h = 0; h < 8; ++h) {
+                    if (h >= p.G) break;
+                    const float dsh = __shfl_sync(0xffffffffu, dl[h], (k1 + u) & 31);
+                    if (cc[u] < 0) continue;
+#pragma unroll
+                    for (int r = 0; r < DL; ++r) acc[h][r] = fmaf(dsh, kv[u][r], acc[h][r]);
+                }
+            }
         }
     }
 #pragma unroll
@@ -156,6 +202,11 @@ __global__ void __launch_bounds__(128) bwd_dqs_kernel(const BwdRowsParams p) {
 }
 
 // ---------------------------------------------------------------- rows
+// Two CTAs share an SM: TMEM holds dQ (D columns) and S, U of one tile (64
+// columns each) within 256 columns, shared memory Q, dO and one stage each of
+// K and V; each CTA's softmax covers the other's MMA and copy latencies. K of
+// a pass-A tile is handed back when its S product is done, of a pass-B tile
+// when its dQ product is; V when its U product is.
 template <int D>
 struct RowLayout {
     static constexpr uint32_t Q_BYTES = kRows * D * 2;        // Q or dO rows
@@ -163,20 +214,17 @@ struct RowLayout {
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_O = Q_BYTES;                // dO
     static constexpr uint32_t OFF_K = 2 * Q_BYTES;
-    static constexpr uint32_t OFF_V = OFF_K + kRStg * KV_BYTES;
-    static constexpr uint32_t OFF_SMALL = OFF_V + kRStg * KV_BYTES;
-    // TMEM: dQ [0, D); buffer sb: S at BUF + 128 sb, U at BUF + 128 sb + 64
-    static constexpr int TM_DQ = 0, TM_BUF = D;
-    static constexpr uint32_t TMEM_COLS = 512u;
+    static constexpr uint32_t OFF_V = OFF_K + KV_BYTES;
+    static constexpr uint32_t OFF_SMALL = OFF_V + KV_BYTES;
+    static constexpr int TM_DQ = 0, TM_S = D, TM_U = D + kTile;
+    static constexpr uint32_t TMEM_COLS = 256u;
+    static_assert(D + 2 * kTile <= 256, "TMEM budget of two CTAs per SM");
 };
 
 struct RowSmall {
     uint64_t q_full;
-    uint64_t full[kRStg];
-    uint64_t empty[kRStg];
-    uint64_t s_full[2];
-    uint64_t p_full[2];
-    uint64_t buf_free[2];
+    uint64_t k_full, v_full, k_empty, v_empty;
+    uint64_t s_full, p_full;
     uint64_t acc_done;
     uint32_t tmem_base;
     int abort;
@@ -185,19 +233,19 @@ struct RowSmall {
     int win_start;
 };
 
-__device__ __forceinline__ float row_max64(const uint32_t *r) {
+__device__ __forceinline__ float row_max32(const uint32_t *r) {
     float m[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) m[k] = __uint_as_float(r[k]);
 #pragma unroll
-    for (int j = 4; j < 64; j += 4)
+    for (int j = 4; j < 32; j += 4)
 #pragma unroll
         for (int k = 0; k < 4; ++k) m[k] = fmaxf(m[k], __uint_as_float(r[j + k]));
     return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
 }
 
 template <int D>
-__global__ void __launch_bounds__(kRT, 1)
+__global__ void __launch_bounds__(kRT, 2)
 bwd_rows_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV,
                    const BwdRowsParams p) {
@@ -221,15 +269,12 @@ bwd_rows_tc_kernel(const __grid_constant__ CUtensorMap tmK,
 
     if (threadIdx.x == 0) {
         mbar_init(&st.q_full, 128);
-        for (int s = 0; s < kRStg; ++s) {
-            mbar_init(&st.full[s], 1);
-            mbar_init(&st.empty[s], 1);
-        }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&st.s_full[s], 1);
-            mbar_init(&st.p_full[s], 128);
-            mbar_init(&st.buf_free[s], 1);
-        }
+        mbar_init(&st.k_full, 1);
+        mbar_init(&st.v_full, 1);
+        mbar_init(&st.k_empty, 1);
+        mbar_init(&st.v_empty, 1);
+        mbar_init(&st.s_full, 1);
+        mbar_init(&st.p_full, 4);                   // one arrival per softmax warp
         mbar_init(&st.acc_done, 1);
         st.abort = (p.status && *(volatile int32_t *)p.status ==
                                     HILS_ERR_DEVICE_TIMEOUT) ? 1 : 0;
@@ -304,22 +349,38 @@ bwd_rows_tc_kernel(const __grid_constant__ CUtensorMap tmK,
         if (lane == 0) {
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
-            int n = 0;
-            for (; n < NS; ++n) {
-                const int s = n % kRStg;
-                if (n >= kRStg && !mbar_wait(&st.empty[s], ((n / kRStg) - 1) & 1, abort)) break;
+            auto load = [&](int n, bool is_v) {
+                uint64_t *bar = is_v ? &st.v_full : &st.k_full;
                 const int row = tile_row(n % NT);
-                mbar_expect_tx(&st.full[s], 2 * L::KV_BYTES);
-                for (int dh = 0; dh < D / 64; ++dh) {
-                    tma_load_4d(smem + L::OFF_K + s * L::KV_BYTES + dh * (kTile * 128), &tmK,
-                                &st.full[s], dh * 64, row, g, b);
-                    tma_load_4d(smem + L::OFF_V + s * L::KV_BYTES + dh * (kTile * 128), &tmV,
-                                &st.full[s], dh * 64, row, g, b);
+                mbar_expect_tx(bar, L::KV_BYTES);
+                for (int dh = 0; dh < D / 64; ++dh)
+                    tma_load_4d(smem + (is_v ? L::OFF_V : L::OFF_K) + dh * (kTile * 128),
+                                is_v ? &tmV : &tmK, bar, dh * 64, row, g, b);
+            };
+            // each copy goes as soon as its stage has been handed back
+            int nk = 0, nv = 0;
+            uint64_t t_last = globaltimer();
+            for (uint32_t it = 0; nk < NS || nv < NS; ++it) {
+                if (nk < NS && (nk == 0 || mbar_test(smem_u32(&st.k_empty), (nk - 1) & 1))) {
+                    load(nk++, false);
+                    t_last = globaltimer();
+                    continue;
+                }
+                if (nv < NS && (nv == 0 || mbar_test(smem_u32(&st.v_empty), (nv - 1) & 1))) {
+                    load(nv++, true);
+                    t_last = globaltimer();
+                    continue;
+                }
+                if ((it & 255u) == 0) {
+                    if (*abort) break;
+                    if (globaltimer() - t_last > kWaitLimitNs) { *abort = 1; break; }
                 }
             }
-            if (*abort)
-                for (int t = (n > kRStg ? n - kRStg : 0); t < n; ++t)
-                    mbar_drain(&st.full[t % kRStg], (t / kRStg) & 1);
+            // on abort: let the copies already issued land before exiting
+            if (*abort) {
+                if (nk > 0) mbar_drain(&st.k_full, (nk - 1) & 1);
+                if (nv > 0) mbar_drain(&st.v_full, (nv - 1) & 1);
+            }
         }
     } else if (warp == 1) {
         // ----------------------------------------------------- MMA issuer
@@ -332,49 +393,50 @@ bwd_rows_tc_kernel(const __grid_constant__ CUtensorMap tmK,
             const uint32_t sV = smem_u32(smem + L::OFF_V);
             bool ok = mbar_wait(&st.q_full, 0, abort);
             int ndq = 0;                             // dQ products issued
-            // step u's buffer is released once the softmax warps are done
-            // with it; in pass B after dQ += dS K has consumed dS
-            auto finish = [&](int u) -> bool {
-                const int sb = u & 1, s = u % kRStg;
-                if (!mbar_wait(&st.p_full[sb], (u >> 1) & 1, abort)) return false;
-                tc_fence_after();
-                if (u >= NT) {
+            // dQ += dS K for pass-B step u (dS in the S columns); hands K back
+            auto dq = [&](int u) {
 #pragma unroll
-                    for (int kk = 0; kk < kTile / 16; ++kk) {
-                        const uint64_t bk = desc_sw128(sK + s * L::KV_BYTES + kk * 16 * 128,
-                                                       kTile * 128, 1024);
-                        mma_ts(tmem + L::TM_DQ, tmem + L::TM_BUF + sb * 128 + kk * 8, bk, id_q,
-                               (ndq > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    ++ndq;
+                for (int kk = 0; kk < kTile / 16; ++kk) {
+                    const uint64_t bk = desc_sw128(sK + kk * 16 * 128, kTile * 128, 1024);
+                    mma_ts(tmem + L::TM_DQ, tmem + L::TM_S + kk * 8, bk, id_q,
+                           (ndq > 0 || kk > 0) ? 1u : 0u);
                 }
-                mma_commit(&st.buf_free[sb]);
-                mma_commit(&st.empty[s]);
-                return true;
+                ++ndq;
+                mma_commit(&st.k_empty);
+                (void)u;
             };
             for (int n = 0; ok && n < NS; ++n) {
-                const int s = n % kRStg, sb = n & 1;
-                if (!mbar_wait(&st.full[s], (n / kRStg) & 1, abort)) { ok = false; break; }
-                if (n >= 2 && !mbar_wait(&st.buf_free[sb], ((n >> 1) - 1) & 1, abort)) { ok = false; break; }
+                // the softmax warps are done with step n-1's S / U (and, in
+                // pass B, have left dS for its dQ product)
+                if (n >= 1) {
+                    if (!mbar_wait(&st.p_full, (n - 1) & 1, abort)) { ok = false; break; }
+                    tc_fence_after();
+                    if (n - 1 >= NT) dq(n - 1);
+                }
+                if (!mbar_wait(&st.k_full, n & 1, abort)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t aq = desc_sw128(sQ + (kk / 4) * (kRows * 128) + (kk % 4) * 32, 16, 1024);
-                    const uint64_t bk = desc_sw128(sK + s * L::KV_BYTES + (kk / 4) * (kTile * 128) +
-                                                       (kk % 4) * 32, 16, 1024);
-                    mma_ss(tmem + L::TM_BUF + sb * 128, aq, bk, id_s, kk > 0 ? 1u : 0u);
+                    const uint64_t bk = desc_sw128(sK + (kk / 4) * (kTile * 128) + (kk % 4) * 32, 16, 1024);
+                    mma_ss(tmem + L::TM_S, aq, bk, id_s, kk > 0 ? 1u : 0u);
                 }
+                if (n < NT) mma_commit(&st.k_empty);
+                if (!mbar_wait(&st.v_full, n & 1, abort)) { ok = false; break; }
+                tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t ao = desc_sw128(sO + (kk / 4) * (kRows * 128) + (kk % 4) * 32, 16, 1024);
-                    const uint64_t bv = desc_sw128(sV + s * L::KV_BYTES + (kk / 4) * (kTile * 128) +
-                                                       (kk % 4) * 32, 16, 1024);
-                    mma_ss(tmem + L::TM_BUF + sb * 128 + 64, ao, bv, id_s, kk > 0 ? 1u : 0u);
+                    const uint64_t bv = desc_sw128(sV + (kk / 4) * (kTile * 128) + (kk % 4) * 32, 16, 1024);
+                    mma_ss(tmem + L::TM_U, ao, bv, id_s, kk > 0 ? 1u : 0u);
                 }
-                mma_commit(&st.s_full[sb]);
-                if (n >= 1 && !finish(n - 1)) { ok = false; break; }
+                mma_commit(&st.v_empty);
+                mma_commit(&st.s_full);
             }
-            if (ok) finish(NS - 1);
+            if (ok && mbar_wait(&st.p_full, (NS - 1) & 1, abort)) {
+                tc_fence_after();
+                dq(NS - 1);
+            }
             mma_commit(&st.acc_done);
             mbar_drain(&st.acc_done, 0);
         }
@@ -431,84 +493,79 @@ bwd_rows_tc_kernel(const __grid_constant__ CUtensorMap tmK,
             mbar_arrive(&st.q_full);
         }
 
-        const int *myidx = s_idx + m;                // stride M
+        const int *myidx = s_idx + m;                // stride M; valid slots form a prefix
         const int M_ = p.M;
         const float sl2 = p.inv_sqrt_d * kLog2e;
         const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-        // pass A state: the current chunk's (max, sum, sum * u) in log2
-        // units; the window's
+        // The row's next selected slot kp, its chunk ck, and that slot's
+        // record prefetched (lz, Ubar, -, s^).
+        int kp = 0, ck = 0x7fffffff;
+        float4 rec = make_float4(0.f, 0.f, 0.f, 0.f);
+        // move to the first selected slot at or after k and fetch its record
+        auto seek = [&](int k) {
+            while (valid && k < p.K && myidx[k * M_] < 0) ++k;
+            kp = k;
+            ck = (valid && k < p.K) ? myidx[k * M_] : 0x7fffffff;
+            if (ck != 0x7fffffff) rec = *reinterpret_cast<const float4 *>(cs + k * 4);
+        };
+        seek(0);
+        // pass A: the current chunk's (max, sum, sum * u) and the selected
+        // chunks' running (max, sum of e^s^, sum of e^s^ Ubar), log2 units;
+        // the window's (max, sum, sum * u)
         float cm = -INFINITY, cz = 0.f, czu = 0.f;
+        float rm = -INFINITY, rz = 0.f, rd = 0.f;
         float wm = -INFINITY, wz = 0.f, wzu = 0.f;
-        float Lr = 0.f, Dr = 0.f, L2 = 0.f;
-        int kp = 0;                                  // position in this row's selection
+        float L2 = 0.f, Dr = 0.f;
         float a2 = 0.f, ub = 0.f;                    // pass B: current chunk's a (log2), Ubar
         bool ok = true;
 
         for (int n = 0; n < NS; ++n) {
-            const int sb = n & 1;
             const bool passB = n >= NT;
             const int t = passB ? n - NT : n;
             if (n == NT) {
-                // ---- between the passes: L, D; a_c and dsh_c per slot
+                // ---- between the passes: L, D of the row
                 if (valid) {
-                    float top = wm;                  // the window holds token i
-                    for (int k = 0; k < p.K; ++k)
-                        if (myidx[k * M_] >= 0) top = fmaxf(top, cs[k * 4 + 3] * kLog2e);
-                    float tot = wz * fast_exp2(wm - top);
-                    for (int k = 0; k < p.K; ++k)
-                        if (myidx[k * M_] >= 0) tot += fast_exp2(cs[k * 4 + 3] * kLog2e - top);
+                    const float top = fmaxf(rm, wm);           // the window holds token i
+                    const float tot = (rm == -INFINITY ? 0.f : rz * fast_exp2(rm - top)) +
+                                      wz * fast_exp2(wm - top);
                     L2 = top + __log2f(tot);
-                    float Dv = wzu * fast_exp2(wm - L2);
-                    for (int k = 0; k < p.K; ++k)
-                        if (myidx[k * M_] >= 0) Dv += fast_exp2(cs[k * 4 + 3] * kLog2e - L2) * cs[k * 4 + 1];
-                    Lr = L2 * kLn2;
-                    Dr = Dv;
-                    for (int k = 0; k < p.K; ++k) {
-                        if (myidx[k * M_] < 0) continue;
-                        const float lz = cs[k * 4], ubk = cs[k * 4 + 1], sh = cs[k * 4 + 3];
-                        cs[k * 4] = lz - sh + Lr;
-                        cs[k * 4 + 2] = fast_exp2((sh - Lr) * kLog2e) * (ubk - Dr);
-                    }
-                    p.rowstat[rq * 2] = Lr;
+                    Dr = (rm == -INFINITY ? 0.f : rd * fast_exp2(rm - L2)) + wzu * fast_exp2(wm - L2);
+                    p.rowstat[rq * 2] = L2 * kLn2;
                     p.rowstat[rq * 2 + 1] = Dr;
                 }
-                kp = 0;
+                seek(0);
             }
-            if (!__all_sync(0xffffffffu, mbar_wait(&st.s_full[sb], (n >> 1) & 1, abort))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, mbar_wait(&st.s_full, n & 1, abort))) { ok = false; break; }
             tc_fence_after();
-            const uint32_t tS = trow + L::TM_BUF + sb * 128;
+            const uint32_t tS = trow + L::TM_S, tU = trow + L::TM_U;
             // does this row's query select the tile's chunk (chunk tiles)
-            bool sel = false;
-            bool first = false, last = false;
-            int kslot = 0;
+            bool sel = false, first = false, last = false;
             if (t < U * HT) {
                 const int c = s_union[t / HT];
                 first = (t % HT) == 0;
                 last = (t % HT) == HT - 1;
-                int ck = kp < p.K ? myidx[kp * M_] : 0x7fffffff;
-                while (kp < p.K && (ck < c)) {
-                    ++kp;
-                    ck = kp < p.K ? myidx[kp * M_] : 0x7fffffff;
-                }
-                sel = valid && kp < p.K && ck == c;
-                kslot = kp;
-                if (sel && last) ++kp;
+                if (first)
+                    while (ck < c) seek(kp + 1);         // not ascending: skip
+                sel = ck == c;
             }
-            const int j0 = t - U * HT >= 0 ? wstart + (t - U * HT) * kTile : 0;
             const bool win = t >= U * HT;
+            const int j0 = win ? wstart + (t - U * HT) * kTile : 0;
             const bool edge = win && (!valid || j0 < w0 || j0 + kTile - 1 > i);
             const bool any_edge = __any_sync(0xffffffffu, edge);
-            const bool need = win ? true : __any_sync(0xffffffffu, sel);
+            const bool need = win || __any_sync(0xffffffffu, sel);
             if (!passB) {
                 // ------------------------------------------------ pass A
+                // TMEM loads are warp-collective: every lane of a warp that
+                // needs the tile loads S and U in one round trip; lanes whose
+                // row does not take part discard the sums.
                 if (need) {
                     uint32_t sr[64], ur[64];
                     tmem_ld32(tS, sr);
                     tmem_ld32(tS + 32, sr + 32);
-                    tmem_ld32(tS + 64, ur);
-                    tmem_ld32(tS + 96, ur + 32);
+                    tmem_ld32(tU, ur);
+                    tmem_ld32(tU + 32, ur + 32);
                     tmem_wait_ld();
-                    if (win && any_edge) {
+                    if (any_edge) {
 #pragma unroll
                         for (int j = 0; j < 64; ++j) {
                             const int pos = j0 + j;
@@ -516,66 +573,93 @@ bwd_rows_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                             sr[j] = in ? sr[j] : __float_as_uint(-INFINITY);
                         }
                     }
-                    if (win || sel) {
-                        const float mx = row_max64(sr) * sl2;
-                        float &M = win ? wm : cm;
-                        float &Z = win ? wz : cz;
-                        float &ZU = win ? wzu : czu;
-                        if (!win && first) { M = -INFINITY; Z = 0.f; ZU = 0.f; }
-                        const float mn = fmaxf(M, mx);
-                        if (mn != -INFINITY) {
-                            const float f = fast_exp2(M - mn);
-                            float z4[4] = {0.f, 0.f, 0.f, 0.f}, zu4[4] = {0.f, 0.f, 0.f, 0.f};
+                    const float mx = fmaxf(row_max32(sr), row_max32(sr + 32)) * sl2;
+                    const bool act = win || sel;
+                    if (act && !win && first) { cm = -INFINITY; cz = 0.f; czu = 0.f; }
+                    float &Mv = win ? wm : cm;
+                    float &Zv = win ? wz : cz;
+                    float &ZUv = win ? wzu : czu;
+                    const float mn = fmaxf(Mv, mx);
+                    const bool go = act && mn != -INFINITY;
+                    const float mref = go ? mn : 0.f;
+                    float2 z2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                    float2 zu2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                    const float2 nmn = make_float2(-mref, -mref), sl2v = make_float2(sl2, sl2);
 #pragma unroll
-                            for (int j = 0; j < 64; ++j) {
-                                const float e = fast_exp2(fmaf(__uint_as_float(sr[j]), sl2, -mn));
-                                z4[j & 3] += e;
-                                zu4[j & 3] = fmaf(e, __uint_as_float(ur[j]), zu4[j & 3]);
-                            }
-                            Z = Z * f + ((z4[0] + z4[1]) + (z4[2] + z4[3]));
-                            ZU = ZU * f + ((zu4[0] + zu4[1]) + (zu4[2] + zu4[3]));
-                            M = mn;
-                        }
-                        if (!win && last) {          // lz_c (natural log), Ubar_c
-                            cs[kslot * 4] = (cm + __log2f(cz)) * kLn2;
-                            cs[kslot * 4 + 1] = czu / cz;
-                        }
+                    for (int j = 0; j < 32; ++j) {
+                        // masked scores are -inf: their weights are exp2(-inf) = 0
+                        float2 e = f2_fma(make_float2(__uint_as_float(sr[2 * j]),
+                                                      __uint_as_float(sr[2 * j + 1])), sl2v, nmn);
+                        e.x = fast_exp2(e.x);
+                        e.y = fast_exp2(e.y);
+                        z2[j & 1] = f2_add(z2[j & 1], e);
+                        zu2[j & 1] = f2_fma(e, make_float2(__uint_as_float(ur[2 * j]),
+                                                           __uint_as_float(ur[2 * j + 1])),
+                                            zu2[j & 1]);
+                    }
+                    if (go) {
+                        const float f = fast_exp2(Mv - mn);
+                        Zv = Zv * f + ((z2[0].x + z2[0].y) + (z2[1].x + z2[1].y));
+                        ZUv = ZUv * f + ((zu2[0].x + zu2[0].y) + (zu2[1].x + zu2[1].y));
+                        Mv = mn;
+                    }
+                    if (sel && last) {
+                        // lz_c (natural log), Ubar_c; fold e^s^_c into the
+                        // running sums; move to the next slot
+                        const float ubc = czu / cz;
+                        cs[kp * 4] = (cm + __log2f(cz)) * kLn2;
+                        cs[kp * 4 + 1] = ubc;
+                        const float sh2 = rec.w * kLog2e;
+                        const float nr = fmaxf(rm, sh2);
+                        const float f = rm == -INFINITY ? 0.f : fast_exp2(rm - nr);
+                        const float e = fast_exp2(sh2 - nr);
+                        rz = rz * f + e;
+                        rd = rd * f + e * ubc;
+                        rm = nr;
+                        seek(kp + 1);
                     }
                 }
                 tc_fence_before();
-                mbar_arrive(&st.p_full[sb]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&st.p_full);
             } else {
                 // ------------------------------------------------ pass B
+                if (sel && first) {
+                    // a_c = lz_c - s^_c + L; dsh_c = e^{s^_c - L} (Ubar_c - D)
+                    a2 = (rec.x - rec.w) * kLog2e + L2;
+                    ub = rec.y;
+                    cs[kp * 4] = a2 * kLn2;
+                    cs[kp * 4 + 2] = fast_exp2(rec.w * kLog2e - L2) * (rec.y - Dr);
+                }
+                const float sub = win ? L2 : a2;
+                const float del = win ? Dr : ub;
+                const bool act = win ? valid : sel;
+                const float2 nsub = make_float2(-sub, -sub), ndel = make_float2(-del, -del);
+                const float2 sl2v = make_float2(sl2, sl2);
                 uint32_t pk[32];
                 if (need) {
-                    if (sel && first) {
-                        a2 = cs[kslot * 4] * kLog2e;
-                        ub = cs[kslot * 4 + 1];
-                    }
                     uint32_t sr[64], ur[64];
                     tmem_ld32(tS, sr);
                     tmem_ld32(tS + 32, sr + 32);
-                    tmem_ld32(tS + 64, ur);
-                    tmem_ld32(tS + 96, ur + 32);
+                    tmem_ld32(tU, ur);
+                    tmem_ld32(tU + 32, ur + 32);
                     tmem_wait_ld();
-                    const float sub = win ? L2 : a2;
-                    const float del = win ? Dr : ub;
-                    const bool act = win ? valid : sel;
+                    if (any_edge) {
+#pragma unroll
+                        for (int j = 0; j < 64; ++j) {
+                            const int pos = j0 + j;
+                            const bool in = valid && pos >= w0 && pos <= i;
+                            sr[j] = in ? sr[j] : __float_as_uint(-INFINITY);
+                        }
+                    }
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         float2 e = f2_fma(make_float2(__uint_as_float(sr[2 * j]),
-                                                      __uint_as_float(sr[2 * j + 1])),
-                                          make_float2(sl2, sl2), make_float2(-sub, -sub));
+                                                      __uint_as_float(sr[2 * j + 1])), sl2v, nsub);
                         e.x = fast_exp2(e.x);
                         e.y = fast_exp2(e.y);
-                        if (win && any_edge) {
-                            const int pos = j0 + 2 * j;
-                            e.x = (valid && pos >= w0 && pos <= i) ? e.x : 0.f;
-                            e.y = (valid && pos + 1 >= w0 && pos + 1 <= i) ? e.y : 0.f;
-                        }
                         const float2 du = f2_add(make_float2(__uint_as_float(ur[2 * j]),
-                                                             __uint_as_float(ur[2 * j + 1])),
-                                                 make_float2(-del, -del));
+                                                             __uint_as_float(ur[2 * j + 1])), ndel);
                         const float2 ds = f2_mul(e, du);
                         pk[j] = act ? pack_bf16(ds.x, ds.y) : 0u;
                     }
@@ -583,17 +667,20 @@ bwd_rows_tc_kernel(const __grid_constant__ CUtensorMap tmK,
 #pragma unroll
                     for (int j = 0; j < 32; ++j) pk[j] = 0u;
                 }
+                // dS over S columns [0, 32), already read
                 tmem_st32(tS, pk);
+                if (sel && last) seek(kp + 1);
                 tmem_wait_st();
                 tc_fence_before();
-                mbar_arrive(&st.p_full[sb]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&st.p_full);
             }
         }
         // dQ (through the tokens) once the last product is done
         if (ok && NS > 0) ok = __all_sync(0xffffffffu, mbar_wait(&st.acc_done, 0, abort));
         if (ok) {
             tc_fence_after();
-            float *dq = p.dQ + rq * D;
+            float *dqr = p.dQ + rq * D;
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t rv[32];
@@ -602,7 +689,7 @@ bwd_rows_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                 if (valid) {
 #pragma unroll
                     for (int q = 0; q < 32; q += 4)
-                        *reinterpret_cast<float4 *>(dq + c0 + q) = make_float4(
+                        *reinterpret_cast<float4 *>(dqr + c0 + q) = make_float4(
                             __uint_as_float(rv[q]) * p.inv_sqrt_d, __uint_as_float(rv[q + 1]) * p.inv_sqrt_d,
                             __uint_as_float(rv[q + 2]) * p.inv_sqrt_d, __uint_as_float(rv[q + 3]) * p.inv_sqrt_d);
                 }
@@ -620,14 +707,11 @@ bwd_rows_tc_kernel(const __grid_constant__ CUtensorMap tmK,
     }
 }
 
-// Shared memory of one CTA, at least 116 KB: two CTAs on one SM would
-// contend for its 512 TMEM columns.
 template <int D>
 size_t rows_smem(const BwdRowsParams &p) {
     size_t small = sizeof(RowSmall) + sizeof(int) * ((size_t)p.M * p.K + p.ucap) +
                    sizeof(uint32_t) * (((size_t)p.nC + 31) / 32);
-    const size_t n = 1024 + RowLayout<D>::OFF_SMALL + ((small + 15) / 16) * 16;
-    return n < 116 * 1024 ? 116 * 1024 : n;
+    return 1024 + RowLayout<D>::OFF_SMALL + ((small + 15) / 16) * 16;
 }
 
 template <int D>

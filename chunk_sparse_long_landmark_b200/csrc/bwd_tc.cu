@@ -31,9 +31,9 @@
 // rows select) is cut into work units of that many batches, one CTA each:
 // they write partial sums, and the last unit to finish (an integer ticket)
 // adds them in unit order.
-// Warp roles: warps 0-3 gather producers (16 pairs of each batch apiece;
-// thread 0 also issues the one-time TMA of the K / V block), warps 4-7
-// softmax and epilogue, warp 8 MMA issuer and TMEM owner.
+// Warp roles: warps 0-1 gather producers (32 pairs of each batch apiece;
+// thread 0 also issues the one-time TMA of the K / V block), warps 2-5
+// softmax and epilogue, warp 6 MMA issuer and TMEM owner.
 // Every wait is bounded; a lost arrival ends the kernel with
 // HILS_ERR_DEVICE_TIMEOUT in the status word. No floating-point atomics:
 // each output element is summed in one fixed order.
@@ -55,7 +55,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kProd = 4;          // gather producer warps of the key kernel
+constexpr int kProd = 2;          // gather producer warps of the key kernel
 constexpr int kKT = 32 * (kProd + 4 + 1);   // + 4 softmax warps + the MMA warp
 constexpr int kBlk = 128;         // tokens per CTA
 constexpr int kNP = 64;           // pairs per batch
@@ -287,11 +287,9 @@ struct KeySmall {
     uint32_t tmem_base;
     int abort;
     int last;
-    // per stage and pair: {a, delta, dsh, -} (cp.async), lo | len << 8 |
-    // (chunk slot + 1) << 17
+    // per stage and pair: {a, delta, dsh, -} (cp.async), lo | len << 8
     float4 st4[NSTG][kNP];
     int meta[NSTG][kNP];
-    int cflag[NSTG][kProd];                     // producer warp's pairs hold a chunk role
     float dkl[2][128 / (D / 2)][D];             // partial dk' per chunk and range
     float dbl[2][128 / (D / 2)];                // partial db' per chunk and range
 };
@@ -326,6 +324,9 @@ bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                    const BwdTcParams p) {
     using L = KeyLayout<D, QCAL>;
     constexpr int NSTG = L::NSTG;
+    // A batch is handed over once the next one is issued (LAG = 1): handing
+    // it over later ties its start to the release of an older stage.
+    constexpr int LAG = 1;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     KeySmall<D, NSTG> &st = *reinterpret_cast<KeySmall<D, NSTG> *>(smem + L::OFF_SMALL);
@@ -357,7 +358,7 @@ bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap tmK,
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&st.s_full[s], 1);
-            mbar_init(&st.p_full[s], 128);
+            mbar_init(&st.p_full[s], 4);            // one arrival per softmax warp
             mbar_init(&st.buf_free[s], 1);
         }
         mbar_init(&st.acc_done, 1);
@@ -375,8 +376,8 @@ bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap tmK,
 
     if (warp < kProd) {
         // ----------------------------------------------------- producers
-        // warp pw gathers pairs [16 pw, 16 pw + 16) of every batch; lane l
-        // < 16 resolves pair 16 pw + l
+        // warp pw gathers pairs [32 pw, 32 pw + 32) of every batch; lane l
+        // resolves pair 32 pw + l
         const int pw = warp;
         if (run && threadIdx.x == 0) {
             prefetch_tmap(&tmK);
@@ -392,12 +393,11 @@ bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap tmK,
         const __nv_bfloat16 *Qp = reinterpret_cast<const __nv_bfloat16 *>(p.Q);
         const __nv_bfloat16 *Op = reinterpret_cast<const __nv_bfloat16 *>(p.dO);
         const __nv_bfloat16 *Sp = reinterpret_cast<const __nv_bfloat16 *>(p.Qs);
-        const int pr = pw * 16 + (lane & 15);
-        const bool resolver = lane < 16;
+        const int pr = pw * 32 + lane;
         const int32_t *ent = p.ent + (int64_t)bg * p.ent_stride;
         auto entry_of = [&](int t) -> int {          // index entry of pair pr of batch t
             const int e = (t0 + t) * kNP + pr;
-            if (!resolver || t >= T || e >= w.npairs) return -1;
+            if (t >= T || e >= w.npairs) return -1;
             const int item = e / G;
             if (item >= w.nlist) return -1;
             return __ldg(ent + (item < w.ccount[0] ? w.cstart[0] + item
@@ -414,8 +414,7 @@ bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                 break;
             const int efar = entry_of(t + 2);
             int roff = -1;
-            bool chunk_role = false;
-            if (resolver) {
+            {
                 const int e = (t0 + t) * kNP + pr;
                 const uint32_t dst4 = smem_u32(&st.st4[s][pr]);
                 int meta = 0;                        // len = 0: no token
@@ -427,8 +426,7 @@ bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                         const int i = ecur >> 6, k = ecur & 63;
                         roff = (b * p.Hq + hq) * p.N + i;
                         cp_async16(dst4, p.chunkstat + ((int64_t)roff * p.K + k) * 4, 16);
-                        meta = (cpb == 2 ? 64 * q : 0) | (p.S << 8) | ((q + 1) << 17);
-                        chunk_role = true;
+                        meta = (cpb == 2 ? 64 * q : 0) | (p.S << 8);
                     } else {
                         const int i = base + item - w.nlist;
                         roff = (b * p.Hq + hq) * p.N + i;
@@ -446,20 +444,16 @@ bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                 }
                 st.meta[s][pr] = meta;
             }
-            {
-                const unsigned cm = __ballot_sync(0xffffffffu, chunk_role);
-                if (lane == 0) st.cflag[s][pw] = cm != 0u;
-            }
             uint8_t *stg = smem + L::OFF_STG + s * L::STG_BYTES;
 #pragma unroll
             for (int arr = 0; arr < L::NARR; ++arr) {
                 const __nv_bfloat16 *src = arr == 0 ? Qp : (arr == 1 ? Op : Sp);
 #pragma unroll
-                for (int j = 0; j < 16 / PPI; ++j) {
-                    const int pl = j * PPI + lane / UPR;     // pair within the warp's 16
+                for (int j = 0; j < 32 / PPI; ++j) {
+                    const int pl = j * PPI + lane / UPR;     // pair within the warp's 32
                     const int u = lane % UPR;
                     const int ro = __shfl_sync(0xffffffffu, roff, pl);
-                    const int pp = pw * 16 + pl;
+                    const int pp = pw * 32 + pl;
                     const uint32_t dst = smem_u32(stg + arr * L::ROWS_BYTES + (u >> 3) * (kNP * 128) +
                                                   pp * 128 + (((u & 7) ^ (pp & 7)) << 4));
                     cp_async16(dst, ro >= 0 ? (const void *)(src + (int64_t)ro * D + u * 8)
@@ -468,17 +462,19 @@ bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                 }
             }
             cp_commit();
-            if (t >= 1) {
+            // batch t - LAG's copies have landed: hand it to the MMA warp
+            if (t >= LAG) {
                 cp_wait1();
                 fence_async_smem();
-                mbar_arrive(&st.full[(t - 1) % NSTG]);
+                mbar_arrive(&st.full[(t - LAG) % NSTG]);
             }
             ecur = enx;
             enx = efar;
         }
         cp_wait0();
         fence_async_smem();
-        if (run && t == T) mbar_arrive(&st.full[(T - 1) % NSTG]);
+        if (run && t == T)
+            for (int u = max(T - LAG, 0); u < T; ++u) mbar_arrive(&st.full[u % NSTG]);
     } else if (warp == kProd + 4) {
         // ----------------------------------------------------- MMA issuer
         if (run && lane == 0) {
@@ -555,15 +551,17 @@ bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap tmK,
             }
             tc_fence_after();
             const uint32_t tb = trow + L::TM_BUF + sb * 128;
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-                uint32_t sr[32], ur[32], pk[16], dk[16];
-                tmem_ld32(tb + 32 * hf, sr);
-                tmem_ld32(tb + 64 + 32 * hf, ur);
+            {
+                // S^T and U^T of the 64 pairs in one TMEM round trip
+                uint32_t sr[64], ur[64], pk[32], dk[32];
+                tmem_ld32(tb, sr);
+                tmem_ld32(tb + 32, sr + 32);
+                tmem_ld32(tb + 64, ur);
+                tmem_ld32(tb + 96, ur + 32);
                 tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int e0 = 32 * hf + 2 * j;
+                for (int j = 0; j < 32; ++j) {
+                    const int e0 = 2 * j;
                     const float4 A = st.st4[s][e0], B = st.st4[s][e0 + 1];
                     const int ma = st.meta[s][e0], mb = st.meta[s][e0 + 1];
                     const float2 x = f2_fma(make_float2(__uint_as_float(sr[2 * j]),
@@ -581,36 +579,38 @@ bwd_keys_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                     pk[j] = pack_bf16(pv.x, pv.y);
                     dk[j] = pack_bf16(ds.x, ds.y);
                 }
-                tmem_st16(tb + 16 * hf, pk);
-                tmem_st16(tb + 64 + 16 * hf, dk);
+                // P^T over S^T columns [0, 32), dS^T over U^T columns [0, 32)
+                tmem_st32(tb, pk);
+                tmem_st32(tb + 64, dk);
             }
             tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(&st.p_full[sb]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&st.p_full[sb]);
             // dk' and db' of the chunk-role pairs of this thread's range, from
-            // the gathered scoring rows: branch-free (a pair of the other
-            // chunk, or of the window, adds zero); skipped when no producer
-            // warp of the range saw a chunk-role pair
-            bool any = false;
-#pragma unroll
-            for (int q = 0; q < PPR / 16; ++q) any |= st.cflag[s][rng * (PPR / 16) + q] != 0;
-            if (any) {
+            // the gathered scoring rows. A batch holds, in order, pairs of the
+            // block's first chunk, of its second chunk, then window pairs: the
+            // two boundaries follow from the batch's first pair index.
+            {
+                const int eb = (t0 + t) * kNP;
+                const int b0 = min(max(w.ccount[0] * G - eb, 0), kNP);
+                const int b1 = min(max(w.nlist * G - eb, 0), kNP);
+                const int lo = rng * PPR, hi = lo + PPR;
                 const uint8_t *qs = smem + L::OFF_STG + s * L::STG_BYTES + (QCAL ? 2 : 0) * L::ROWS_BYTES +
                                     (dm >> 6) * (kNP * 128);
                 const int byte = (dm & 63) * 2;
-#pragma unroll 8
-                for (int e = rng * PPR; e < (rng + 1) * PPR; ++e) {
-                    const int cq = st.meta[s][e] >> 17;
+                auto acc = [&](int e, float2 &dk, float &db) {
                     const float dsh = st.st4[s][e].z;
-                    const float f0 = cq == 1 ? dsh : 0.f, f1 = cq == 2 ? dsh : 0.f;
                     const uint32_t wq = *reinterpret_cast<const uint32_t *>(
                         qs + e * 128 + ((((byte >> 4) ^ (e & 7)) << 4) | (byte & 15)));
-                    const float qa = __uint_as_float(wq << 16), qb = __uint_as_float(wq & 0xffff0000u);
-                    dk0.x = fmaf(f0, qa, dk0.x); dk0.y = fmaf(f0, qb, dk0.y);
-                    dk1.x = fmaf(f1, qa, dk1.x); dk1.y = fmaf(f1, qb, dk1.y);
-                    db0 += f0;
-                    db1 += f1;
-                }
+                    dk.x = fmaf(dsh, __uint_as_float(wq << 16), dk.x);
+                    dk.y = fmaf(dsh, __uint_as_float(wq & 0xffff0000u), dk.y);
+                    db += dsh;
+                };
+#pragma unroll 4
+                for (int e = lo; e < min(hi, b0); ++e) acc(e, dk0, db0);
+#pragma unroll 4
+                for (int e = max(lo, b0); e < min(hi, b1); ++e) acc(e, dk1, db1);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&st.empty[s]);

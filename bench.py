@@ -830,28 +830,13 @@ def bench_decode(args, dev, stream, flush, world, max_over_ranks, barrier,
     return out
 
 
-def fp32_alu_peak_tflops():
-    """FP32 FMA peak of the CUDA cores from unit counts and clocks: SMs x 128
-    FP32 lanes x 2 FLOP per FMA x the maximum SM clock."""
-    import torch
-    props = torch.cuda.get_device_properties(torch.cuda.current_device())
-    mhz = 1965.0
-    try:
-        import pynvml as nv
-        nv.nvmlInit()
-        h = nv.nvmlDeviceGetHandleByIndex(0)
-        mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
-    except Exception:
-        pass
-    return props.multi_processor_count * 128 * 2 * mhz * 1e6 / 1e12
-
-
 def bench_backward(args, dev, stream, flush, max_over_ranks, barrier, rank):
     """Backward of the 32K prefill workload (selection from the forward,
-    dO ~ N(0,1)), L2 flushed before every call. The kernels run on the CUDA
-    cores in f32: roofline "alu" against the FP32 FMA peak, on the touched
-    FLOPs: 10d per (row, head, attended token) -- s, u, dq, dK, dV -- plus
-    4d per (row, head, selected chunk) for dqs and dk'."""
+    dO ~ N(0,1)), L2 flushed before every call. Its contractions (s, u, dq,
+    dK, dV) run on the tensor cores in bf16 with f32 accumulation: roofline
+    "tensor" against the measured bf16 peak, on the touched FLOPs: 10d per
+    (row, head, attended token) plus 4d per (row, head, selected chunk) for
+    dqs and dk'."""
     import torch
 
     import chunk_sparse_long_landmark_b200 as hils
@@ -896,7 +881,8 @@ def bench_backward(args, dev, stream, flush, max_over_ranks, barrier, rank):
     toks = sel * sh.S + (i - w0 + 1)
     flops = float(sh.B * sh.Hq * sh.d * (10 * toks.sum() + 4 * sel.sum()))
     ach = flops / (ms * 1e-3) / 1e12
-    peak = fp32_alu_peak_tflops()
+    peaks = measured_peaks()
+    peak = peaks["bf16"]
     del inp, idx, dO, grads
     torch.cuda.empty_cache()
     return {"workload": "prefill_32k_backward",
@@ -904,14 +890,18 @@ def bench_backward(args, dev, stream, flush, max_over_ranks, barrier, rank):
                            "forward's selection",
             "value": sh.B * sh.N / (ms * 1e-3), "unit": "tokens/s",
             "ms_per_step": ms, "steps": steps,
-            "roofline": {"bound": "alu", "achieved": ach, "peak": peak,
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": peak,
                          "unit": "TFLOP/s", "frac": ach / peak,
-                         "peak_source": "SMs x 128 FP32 lanes x 2 x max SM clock",
+                         "peak_source": ("measured (burst bf16 GEMM)"
+                                         if peaks["src"] == "measured"
+                                         else "fallback (burst bf16)"),
                          "algorithmic_flops_per_call": flops,
                          "traffic": None},
             "config": {"B": sh.B, "Hq": sh.Hq, "Hkv": sh.Hkv, "d": sh.d,
                        "N": sh.N, "S": sh.S, "W": sh.W, "K": sh.K,
-                       "dtype": "bf16 inputs, f32 arithmetic and gradients",
+                       "dtype": "bf16 inputs; bf16 tensor-core products (p and "
+                                "ds rounded to bf16), f32 accumulation, f32 "
+                                "gradients",
                        "l2": "flushed before every call"}}
 
 

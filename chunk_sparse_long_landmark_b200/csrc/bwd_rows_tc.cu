@@ -68,63 +68,88 @@ __device__ __forceinline__ void load_bf16s(const __nv_bfloat16 *src, float *f) {
 }
 
 // ------------------------------------------------------------------ s^_c
-// Warp per (b, g, i): the row's top-K slots are read 32 at a time (lane =
-// slot) and broadcast; four landmark rows are in flight at once; lanes
-// split the dims of the dot products.
+// Lanes over top-K slots: a lane takes one (row, slot) and forms the whole
+// dot products of the slot's landmark key with the G scoring rows, which
+// the warp first stages in shared memory as f32 (no cross-lane reductions).
+// With K <= 16 a warp takes two rows (16 lanes each), with K > 32 a lane
+// takes two slots.
+constexpr int kShWarps = 4;
+
 template <int D>
-__global__ void __launch_bounds__(128) bwd_sh_kernel(const BwdRowsParams p) {
-    constexpr int DL = D / 32;
+__global__ void __launch_bounds__(32 * kShWarps) bwd_sh_kernel(const BwdRowsParams p) {
+    __shared__ __align__(16) float qsm[kShWarps][2][8][D];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * 4 + warp;      // (b, g, i)
-    if (row >= (int64_t)p.B * p.Hkv * p.N) return;
-    const int i = (int)(row % p.N);
-    const int g = (int)((row / p.N) % p.Hkv);
-    const int b = (int)(row / ((int64_t)p.N * p.Hkv));
-    const int64_t bg = (int64_t)b * p.Hkv + g;
+    const int rpw = p.K <= 16 ? 2 : 1;               // rows per warp
+    const int lpr = 32 / rpw;                        // lanes per row
+    const int64_t nrows = (int64_t)p.B * p.Hkv * p.N;
+    const int64_t row0 = ((int64_t)blockIdx.x * kShWarps + warp) * rpw;
+    if (row0 >= nrows) return;
     const __nv_bfloat16 *Qs = reinterpret_cast<const __nv_bfloat16 *>(p.Qs ? p.Qs : p.Q);
     const __nv_bfloat16 *Kl = reinterpret_cast<const __nv_bfloat16 *>(p.Klm);
+    // stage the scoring rows of the warp's rows (f32), 8 values per lane step
+    for (int e = lane; e < rpw * p.G * (D / 8); e += 32) {
+        const int rs = e / (p.G * (D / 8)), h = (e / (D / 8)) % p.G, u = e % (D / 8);
+        const int64_t row = row0 + rs;
+        float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (row < nrows) {
+            const int i = (int)(row % p.N), g = (int)((row / p.N) % p.Hkv);
+            const int b = (int)(row / ((int64_t)p.N * p.Hkv));
+            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(
+                Qs + (((int64_t)b * p.Hq + p.group_heads[g * p.G + h]) * p.N + i) * D) + u);
+            const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                f[2 * k] = __uint_as_float(x[k] << 16);
+                f[2 * k + 1] = __uint_as_float(x[k] & 0xffff0000u);
+            }
+        }
+        float4 *dst = reinterpret_cast<float4 *>(&qsm[warp][rs][h][u * 8]);
+        dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+        dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
+    __syncwarp();
+    const int rs = lane / lpr;
+    const int64_t row = row0 + rs;
+    if (row >= nrows) return;
+    const int i = (int)(row % p.N), g = (int)((row / p.N) % p.Hkv);
+    const int b = (int)(row / ((int64_t)p.N * p.Hkv));
+    const int64_t bg = (int64_t)b * p.Hkv + g;
     int64_t w0, nc;
     window_bounds(i, p.S, p.W, &w0, &nc);
-    float q[8][DL];
+    for (int k = lane % lpr; k < p.K; k += lpr) {
+        const int c = __ldg(p.idx + (bg * p.N + i) * p.K + k);
+        if (c < 0 || c >= nc) continue;
+        const uint4 *kr = reinterpret_cast<const uint4 *>(Kl + (bg * p.nC + c) * D);
+        float acc[8];
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
-        if (h >= p.G) break;
-        load_bf16s<DL>(Qs + (((int64_t)b * p.Hq + p.group_heads[g * p.G + h]) * p.N + i) * D + lane * DL,
-                       q[h]);
-    }
-    const int32_t *ir = p.idx + (bg * p.N + i) * p.K;
-    for (int k0 = 0; k0 < p.K; k0 += 32) {
-        int cl = k0 + lane < p.K ? __ldg(ir + k0 + lane) : -1;
-        if (cl >= nc) cl = -1;
-        const int kn = min(32, p.K - k0);
-        for (int k1 = 0; k1 < kn; k1 += 4) {
-            float kv[4][DL], bc[4];
-            int cc[4];
+        for (int h = 0; h < 8; ++h) acc[h] = 0.f;
+#pragma unroll 4
+        for (int u = 0; u < D / 8; ++u) {
+            const uint4 w = __ldg(kr + u);
+            const uint32_t x[4] = {w.x, w.y, w.z, w.w};
+            float kv[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                cc[u] = __shfl_sync(0xffffffffu, cl, (k1 + u) & 31);
-                if (k1 + u >= kn) cc[u] = -1;
-                const int c = cc[u] < 0 ? 0 : cc[u];
-                load_bf16s<DL>(Kl + (bg * p.nC + c) * D + lane * DL, kv[u]);
-                bc[u] = __ldg(p.bias + bg * p.nC + c);
+            for (int q = 0; q < 4; ++q) {
+                kv[2 * q] = __uint_as_float(x[q] << 16);
+                kv[2 * q + 1] = __uint_as_float(x[q] & 0xffff0000u);
             }
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (cc[u] < 0) continue;             // uniform over the warp
-#pragma unroll
-                for (int h = 0; h < 8; ++h) {
-                    if (h >= p.G) break;
-                    float a = 0.f;
-#pragma unroll
-                    for (int r = 0; r < DL; ++r) a = fmaf(q[h][r], kv[u][r], a);
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-                    if (lane == 0) {
-                        const int64_t rq = ((int64_t)b * p.Hq + p.group_heads[g * p.G + h]) * p.N + i;
-                        p.chunkstat[(rq * p.K + k0 + k1 + u) * 4 + 3] = a * p.inv_sqrt_d + bc[u];
-                    }
-                }
+            for (int h = 0; h < 8; ++h) {
+                if (h >= p.G) break;
+                const float4 qa = *reinterpret_cast<const float4 *>(&qsm[warp][rs][h][u * 8]);
+                const float4 qb = *reinterpret_cast<const float4 *>(&qsm[warp][rs][h][u * 8 + 4]);
+                acc[h] = fmaf(qa.x, kv[0], acc[h]); acc[h] = fmaf(qa.y, kv[1], acc[h]);
+                acc[h] = fmaf(qa.z, kv[2], acc[h]); acc[h] = fmaf(qa.w, kv[3], acc[h]);
+                acc[h] = fmaf(qb.x, kv[4], acc[h]); acc[h] = fmaf(qb.y, kv[5], acc[h]);
+                acc[h] = fmaf(qb.z, kv[6], acc[h]); acc[h] = fmaf(qb.w, kv[7], acc[h]);
             }
+        }
+        const float bc = __ldg(p.bias + bg * p.nC + c);
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+            if (h >= p.G) break;
+            const int64_t rq = ((int64_t)b * p.Hq + p.group_heads[g * p.G + h]) * p.N + i;
+            p.chunkstat[(rq * p.K + k) * 4 + 3] = acc[h] * p.inv_sqrt_d + bc;
         }
     }
 }
@@ -722,7 +747,8 @@ cudaError_t launch_rows_tc_t(const BwdRowsParams &p, cudaStream_t st) {
         return cudaErrorInvalidValue;
     const int64_t rows = (int64_t)p.B * p.Hkv * p.N;
     const unsigned wgrid = (unsigned)((rows + 3) / 4);
-    if (p.nC > 0) bwd_sh_kernel<D><<<wgrid, 128, 0, st>>>(p);
+    const int64_t sh_rows = (int64_t)kShWarps * (p.K <= 16 ? 2 : 1);
+    if (p.nC > 0) bwd_sh_kernel<D><<<(unsigned)((rows + sh_rows - 1) / sh_rows), 32 * kShWarps, 0, st>>>(p);
     const size_t smem = rows_smem<D>(p);
     auto kern = bwd_rows_tc_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

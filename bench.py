@@ -599,6 +599,8 @@ def main():
                     help="skip the other prefill workloads' legs")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode step (prints its object)")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the 32K prefill backward (prints its object)")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="run the headline workload at this sequence length "
                          "instead of its own (reduced cases for profilers)")
@@ -626,6 +628,13 @@ def main():
     peaks = measured_peaks()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    if args.backward_only:
+        bw = bench_backward(args, dev, stream, flush, max_over_ranks, barrier,
+                            rank)
+        if rank == 0:
+            print(json.dumps({"backward": bw}), flush=True)
+        ranks.close()
+        return
     if args.decode_only:
         d = bench_decode(args, dev, stream, flush, world, max_over_ranks,
                          barrier, rank, peaks)
@@ -896,7 +905,12 @@ def bench_backward(args, dev, stream, flush, max_over_ranks, barrier, rank):
                                          if peaks["src"] == "measured"
                                          else "fallback (burst bf16)"),
                          "algorithmic_flops_per_call": flops,
-                         "traffic": None},
+                         "traffic": profiled_traffic(
+                             ["bwd_rows_tc", "bwd_dqs", "bwd_keys_tc"],
+                             "prefill_32k_backward"),
+                         "traffic_covers": "bwd_rows_tc + bwd_dqs + bwd_keys_tc "
+                                           "(94% of the call; the landmark-score "
+                                           "and index kernels not captured)"},
             "config": {"B": sh.B, "Hq": sh.Hq, "Hkv": sh.Hkv, "d": sh.d,
                        "N": sh.N, "S": sh.S, "W": sh.W, "K": sh.K,
                        "dtype": "bf16 inputs; bf16 tensor-core products (p and "

@@ -285,11 +285,18 @@ hils_status hils_fwd_decode_multi(const hils_decode_multi_args *args, void *stre
  *   given exactly when Qs is; without Qs the scoring gradient is in dQ), dK,
  *   dV [B,Hkv,N,d], dKlm [B,Hkv,nC,d], dbias [B,Hkv,nC].
  *   workspace >= hils_bwd_prefill_workspace_size (per (row, head) and
- *   (row, head, selected chunk) softmax statistics).
- * Deterministic: no floating-point atomics; every output element is summed
- * by one thread in a fixed order. Supported: d in {64,128}, S in {64,128},
- * G = Hq/Hkv <= 8; other shapes return HILS_ERR_UNSUPPORTED. Two kernel
- * launches on `stream`.
+ *   (row, head, selected chunk) softmax statistics; for bf16, also the
+ *   chunk -> (row, slot) index of the selection and the key side's work
+ *   units with room for their partial sums).
+ *   status: device int32, nullable; a kernel whose bounded wait gave up
+ *   writes HILS_ERR_DEVICE_TIMEOUT there (the gradients are then undefined).
+ * bf16 runs on the tensor cores (products of bf16 operands -- the weights
+ * p_j and ds_j are rounded to bf16 -- with f32 accumulation), f32 on the
+ * CUDA cores in f32. Deterministic: no floating-point atomics; every output
+ * element is summed in one fixed order, so repeated calls are bitwise equal.
+ * Supported: d in {64,128}, S in {64,128}, G = Hq/Hkv <= 8; other shapes
+ * return HILS_ERR_UNSUPPORTED. Kernel launches on `stream`: 8 for bf16
+ * (7 when N < S), 2 for f32.
  */
 typedef struct {
     int32_t dtype;

@@ -295,8 +295,8 @@ hils_status hils_fwd_decode_multi(const hils_decode_multi_args *args, void *stre
  * CUDA cores in f32. Deterministic: no floating-point atomics; every output
  * element is summed in one fixed order, so repeated calls are bitwise equal.
  * Supported: d in {64,128}, S in {64,128}, G = Hq/Hkv <= 8; other shapes
- * return HILS_ERR_UNSUPPORTED. Kernel launches on `stream`: 8 for bf16
- * (7 when N < S), 2 for f32.
+ * return HILS_ERR_UNSUPPORTED. Kernel launches on `stream`: at most 8 for
+ * bf16, 2 for f32.
  */
 typedef struct {
     int32_t dtype;

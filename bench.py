@@ -599,6 +599,9 @@ def main():
                     help="skip the other prefill workloads' legs")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode step (prints its object)")
+    ap.add_argument("--decode-batch", type=int, default=0,
+                    help="run the decode legs with this many sequences instead "
+                         "of the workload's (reduced cases for profilers)")
     ap.add_argument("--backward-only", action="store_true",
                     help="time only the 32K prefill backward (prints its object)")
     ap.add_argument("--seq-len", type=int, default=0,
@@ -757,6 +760,9 @@ def bench_decode(args, dev, stream, flush, world, max_over_ranks, barrier,
     import synth
     name, cid = DECODE_WORKLOAD
     sh = synth.DECODE_CONFIGS[cid]
+    if getattr(args, "decode_batch", 0):
+        sh = sh.with_(B=args.decode_batch)
+        name = f"{name}_reduced_b{args.decode_batch}"
     inp = synth.make_decode(sh, seed=synth.seed_for(cid) + 17 * rank,
                             device=dev)
     O = torch.empty_like(inp["Q"])
@@ -811,13 +817,43 @@ def bench_decode(args, dev, stream, flush, world, max_over_ranks, barrier,
         e[2].record(cur)
         torch.cuda.synchronize()
         ss.append((e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])))
+    # end to end through the C ABI: the step's queries copied in from pinned
+    # host memory and O, idx copied back, inside the timed region (the KV
+    # cache and landmarks are resident state)
+    hq = torch.empty(inp["Q"].shape, dtype=inp["Q"].dtype).pin_memory()
+    hq.copy_(inp["Q"].cpu())
+    hO = torch.empty(O.shape, dtype=O.dtype).pin_memory()
+    hidx = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    dq = torch.empty_like(inp["Q"])
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True)
+        hils.fwd_decode(dq, inp["K"], inp["V"], inp["Klm"], inp["bias"],
+                        inp["cache_len"], inp["head_map"], sh.S, sh.W, sh.K,
+                        out=O, idx=idx, sel_score=sel, workspace=ws,
+                        stream=cur)
+        hO.copy_(O, non_blocking=True)
+        hidx.copy_(idx, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    ee = [(torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ee:
+        flush.zero_()
+        a.record(cur)
+        e2e_step()
+        b.record(cur)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ee)) / steps
     cl = inp["cache_len"].cpu().tolist()
     nbytes = decode_bytes(sh, cl)
     ach = nbytes / (ms * 1e-3) / 1e9
     del g
     out = {
         "workload": name, "value": ms * 1e3, "unit": "us/step",
-        "note": "one decode step = one new token for each of the B=8 "
+        "note": f"one decode step = one new token for each of the B={sh.B} "
                 "sequences (per-token latency of every sequence)",
         "median_us": med * 1e3, "tokens_per_s": world * sh.B / (ms * 1e-3),
         "stages_ms": {"select": statistics.mean(x[0] for x in ss),
@@ -826,15 +862,20 @@ def bench_decode(args, dev, stream, flush, world, max_over_ranks, barrier,
                      "achieved": ach, "peak": peaks["hbm"], "unit": "GB/s",
                      "frac": ach / peaks["hbm"], "peak_source": peaks["src"],
                      "algorithmic_bytes_per_step": nbytes,
-                     "traffic": profiled_traffic(["dec_score", "dec_attend"],
-                                                 name),
-                     "traffic_covers": "dec_score + dec_attend launches "
-                                       "(dec_select not captured)"},
+                     "traffic": profiled_traffic(
+                         ["dec_score", "dec_select", "dec_attend"], name),
+                     "traffic_covers": "dec_score + dec_select + dec_attend "
+                                       "launches"},
+        "e2e": {"value": e2e_ms * 1e3, "unit": "us/step",
+                "h2d_bytes_per_step": hq.numel() * hq.element_size(),
+                "d2h_bytes_per_step": hO.numel() * hO.element_size() +
+                                      hidx.numel() * hidx.element_size(),
+                "note": "queries in, O and idx out per step; caches resident"},
         "config": {"B": sh.B, "Hq": sh.Hq, "Hkv": sh.Hkv, "d": sh.d,
                    "L": sh.N, "S": sh.S, "W": sh.W, "K": sh.K,
                    "l2": "flushed before every timed step"},
     }
-    del inp, O, idx, sel, ws
+    del inp, O, idx, sel, ws, dq
     torch.cuda.empty_cache()
     return out
 
@@ -935,6 +976,8 @@ def bench_decode_multi(args, dev, stream, flush, world, max_over_ranks,
     import synth
     name, cid = DECODE_WORKLOAD
     sh = synth.DECODE_CONFIGS[cid]
+    if getattr(args, "decode_batch", 0):
+        sh = sh.with_(B=args.decode_batch)
     T = DECODE_MULTI_T
     inp = synth.make_decode(sh, seed=synth.seed_for(cid) + 17 * rank + 5,
                             device=dev)

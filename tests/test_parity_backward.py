@@ -73,6 +73,9 @@ CASES = {
                                       "qcal"),
     # G = 8: eight pairs per row in a batch of 64
     "bf16_g8_d128": synth.Shape("bf16", 1, 8, 1, 128, 1000, 64, 128, 5),
+    # G = 3 (128 % G != 0): the query side runs on the CUDA cores and feeds
+    # the tensor-core key side
+    "bf16_g3_d64": synth.Shape("bf16", 1, 6, 2, 64, 1100, 64, 160, 5),
     # many key blocks, rows selecting a chunk spread over several batches
     "bf16_g4_d128_long": synth.Shape("bf16", 1, 4, 1, 128, 3000, 64, 128, 12),
 }

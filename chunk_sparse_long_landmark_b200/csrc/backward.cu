@@ -664,6 +664,9 @@ bool keys_tc_ok(const hils_backward_args *a, int G, int nC) {
     if (!(a->S == 64 || a->S == 128) || G > 8 || a->K > 64) return false;
     if (a->N >= (1 << 25) || (size_t)nC * sizeof(int) > 200 * 1024) return false;
     if ((int64_t)a->B * a->Hq * a->N >= (1ll << 31)) return false;
+    // the key side's grid is an upper bound on its work units
+    if (bwd_keys_max_units(a->B, a->Hkv, a->N, a->S, a->W, a->K, G) >= (1ll << 31))
+        return false;
     if (bwd_keys_tc_smem(a->d, a->Qs != nullptr) > 227 * 1024) return false;
     return tc_maps_available();
 }

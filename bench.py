@@ -602,6 +602,9 @@ def main():
     ap.add_argument("--decode-batch", type=int, default=0,
                     help="run the decode legs with this many sequences instead "
                          "of the workload's (reduced cases for profilers)")
+    ap.add_argument("--backward-workload", default="prefill_32k",
+                    choices=sorted(WORKLOADS),
+                    help="prefill workload of the backward leg")
     ap.add_argument("--backward-only", action="store_true",
                     help="time only the 32K prefill backward (prints its object)")
     ap.add_argument("--seq-len", type=int, default=0,
@@ -881,8 +884,9 @@ def bench_decode(args, dev, stream, flush, world, max_over_ranks, barrier,
 
 
 def bench_backward(args, dev, stream, flush, max_over_ranks, barrier, rank):
-    """Backward of the 32K prefill workload (selection from the forward,
-    dO ~ N(0,1)), L2 flushed before every call. Its contractions (s, u, dq,
+    """Backward of a prefill workload (32K unless --backward-workload says
+    otherwise; selection from the forward, dO ~ N(0,1)), L2 flushed before
+    every call. Its contractions (s, u, dq,
     dK, dV) run on the tensor cores in bf16 with f32 accumulation: roofline
     "tensor" against the measured bf16 peak, on the touched FLOPs: 10d per
     (row, head, attended token) plus 4d per (row, head, selected chunk) for
@@ -891,7 +895,8 @@ def bench_backward(args, dev, stream, flush, max_over_ranks, barrier, rank):
 
     import chunk_sparse_long_landmark_b200 as hils
     import synth
-    cid = WORKLOADS["prefill_32k"]
+    wl = getattr(args, "backward_workload", "prefill_32k")
+    cid = WORKLOADS[wl]
     sh = synth.PREFILL_CONFIGS[cid]
     inp = synth.make_prefill(sh, seed=synth.seed_for(cid) + 17 * rank + 3,
                              device=dev)
@@ -935,7 +940,7 @@ def bench_backward(args, dev, stream, flush, max_over_ranks, barrier, rank):
     peak = peaks["bf16"]
     del inp, idx, dO, grads
     torch.cuda.empty_cache()
-    return {"workload": "prefill_32k_backward",
+    return {"workload": f"{wl}_backward",
             "description": "dQ, dK, dV, dk', db' of the 32K prefill for the "
                            "forward's selection",
             "value": sh.B * sh.N / (ms * 1e-3), "unit": "tokens/s",
@@ -948,7 +953,7 @@ def bench_backward(args, dev, stream, flush, max_over_ranks, barrier, rank):
                          "algorithmic_flops_per_call": flops,
                          "traffic": profiled_traffic(
                              ["bwd_rows_tc", "bwd_dqs", "bwd_keys_tc"],
-                             "prefill_32k_backward"),
+                             f"{wl}_backward"),
                          "traffic_covers": "bwd_rows_tc + bwd_dqs + bwd_keys_tc "
                                            "(94% of the call; the landmark-score "
                                            "and index kernels not captured)"},

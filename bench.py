@@ -941,8 +941,8 @@ def bench_backward(args, dev, stream, flush, max_over_ranks, barrier, rank):
     del inp, idx, dO, grads
     torch.cuda.empty_cache()
     return {"workload": f"{wl}_backward",
-            "description": "dQ, dK, dV, dk', db' of the 32K prefill for the "
-                           "forward's selection",
+            "description": f"dQ, dK, dV, dk', db' of the {wl} prefill for "
+                           "the forward's selection",
             "value": sh.B * sh.N / (ms * 1e-3), "unit": "tokens/s",
             "ms_per_step": ms, "steps": steps,
             "roofline": {"bound": "tensor", "achieved": ach, "peak": peak,
